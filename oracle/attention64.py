@@ -1,0 +1,188 @@
+"""FP64 CPU oracle for BF16 attention with the repeated-max fix.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  The product path (the
+CUDA library and its Python binding) never calls it, and it shares no code with
+that path: plain NumPy, whole N x N matrices, one (batch, head) pair at a time.
+
+What it computes, and where each step is stated:
+
+* Standard attention, the "baseline attention" of "Is Flash Attention Stable?"
+  (chibakuma.com; sections "Flash Attention: from academic breakthrough to
+  industry standard" and "What did Meta's study find?"):
+  S = scale * Q K^T, P = softmax(S) per row, O = P V.  Computed here in FP64
+  instead of FP32.  Causal masking (key j visible to query i iff j <= i) is the
+  plain reading for decoder training (GPT-2 and Llama 2 on the pages).
+* The log-sum-exp LSE_i = log sum_j exp(S_ij), the per-row statistic the
+  recomputing backward pass needs (yicaiai article, abstract and section 5.1).
+* The backward pass, written out from the chain rule of the definition above:
+  dV = P^T dO, dP = dO V^T, D_i = sum_k dO_ik O_ik, dS = P * (dP - D),
+  dQ = scale dS K, dK = scale dS^T Q (the gradients d loss/dQ, d loss/dK named
+  in the yicaiai article, section 4.3).
+* The safe-softmax shift and the BF16 rounding point of the unnormalised
+  output ("Why Low-Precision Transformer Training Fails", admirer.cn summary,
+  "mechanism 2"): P_bar = bf16(exp(S - m)), O = (P_bar V) / l.
+* The fix (same section): per row, detect whether the maximum of S occurs more
+  than once; if so raise the shift m so that every exponent, the ones at the
+  maximum included, is strictly below 1.  Reading taken here (the pages leave
+  the amount open): m' = m + delta with delta = -ln(1 - 2^-8), so the maxima
+  map to exactly 1 - 2^-8 = 0.99609375, the largest bf16 value below 1.
+
+Parity pins for every function live in tests/test_oracle_pins.py (brute force,
+closed forms, invariants, finite differences, torch's bf16 cast).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "DELTA_LOG2", "DELTA_NAT", "bf16_round", "scores", "attention_fwd",
+    "attention_bwd", "attention_fwd_bf16p", "tie_counts",
+]
+
+# Shift added to m on repeated-max rows, in log2 units and in natural-log units.
+DELTA_LOG2 = -np.log2(1.0 - 2.0 ** -8)
+DELTA_NAT = -np.log(1.0 - 2.0 ** -8)
+
+_BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
+
+
+def bf16_round(x) -> np.ndarray:
+    """Round to the nearest bf16 value, ties to even, returned as float64.
+
+    bf16 keeps 8 significant bits and the float32 exponent range: the quantum
+    of a normal value in [2^(e-1), 2^e) is 2^(e-8); below 2^-126 the quantum
+    is fixed at 2^-133 (subnormals).  Results beyond the largest finite bf16
+    value become infinities; NaN stays NaN; the sign of zero is kept.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = x.copy()
+    fin = np.isfinite(x) & (x != 0.0)
+    xf = x[fin]
+    _, e = np.frexp(xf)
+    q_exp = np.maximum(e, -125) - 8
+    r = np.ldexp(np.rint(np.ldexp(xf, -q_exp)), q_exp)
+    r = np.where(np.abs(r) > _BF16_MAX, np.copysign(np.inf, xf), r)
+    # keep the sign of values that round to zero
+    r = np.where(r == 0.0, np.copysign(0.0, xf), r)
+    out[fin] = r
+    return out
+
+
+def _f64(a) -> np.ndarray:
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu").double().numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+def _mask(n: int, causal: bool) -> np.ndarray:
+    """True where key j is visible to query i."""
+    if not causal:
+        return np.ones((n, n), dtype=bool)
+    return np.tril(np.ones((n, n), dtype=bool))
+
+
+def scores(q, k) -> np.ndarray:
+    """Raw dot products Q K^T of one head, float64 [N, N] (no scale, no mask)."""
+    return _f64(q) @ _f64(k).T
+
+
+def _heads(*arrays):
+    """Iterate over (b, h) for arrays shaped [B, H, N, d] (or [B, H, N])."""
+    B, H = arrays[0].shape[:2]
+    for b in range(B):
+        for h in range(H):
+            yield b, h
+
+
+def attention_fwd(q, k, v, causal: bool, scale: float):
+    """Exact attention: O [B,H,N,d] and LSE [B,H,N] (natural log), float64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    o = np.empty((B, H, N, v.shape[-1]))
+    lse = np.empty((B, H, N))
+    vis = _mask(N, causal)
+    for b, h in _heads(q):
+        s = scale * (q[b, h] @ k[b, h].T)
+        s = np.where(vis, s, -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        l = e.sum(axis=1, keepdims=True)
+        p = e / l
+        o[b, h] = p @ v[b, h]
+        lse[b, h] = m[:, 0] + np.log(l[:, 0])
+    return o, lse
+
+
+def attention_bwd(q, k, v, do, causal: bool, scale: float):
+    """Exact gradients (dQ, dK, dV) of sum(dO * O) for O = attention(Q, K, V)."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, N, d = q.shape
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    vis = _mask(N, causal)
+    for b, h in _heads(q):
+        s = scale * (q[b, h] @ k[b, h].T)
+        s = np.where(vis, s, -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        p = e / e.sum(axis=1, keepdims=True)
+        o = p @ v[b, h]
+        dv[b, h] = p.T @ do[b, h]
+        dp = do[b, h] @ v[b, h].T
+        D = np.sum(do[b, h] * o, axis=1, keepdims=True)
+        ds = p * (dp - D)
+        dq[b, h] = scale * (ds @ k[b, h])
+        dk[b, h] = scale * (ds.T @ q[b, h])
+    return dq, dk, dv
+
+
+def tie_counts(q, k, causal: bool) -> np.ndarray:
+    """Per row, how many visible keys reach the row maximum of S exactly (int64 [B,H,N])."""
+    q, k = _f64(q), _f64(k)
+    B, H, N, _ = q.shape
+    out = np.empty((B, H, N), dtype=np.int64)
+    vis = _mask(N, causal)
+    for b, h in _heads(q):
+        s = np.where(vis, q[b, h] @ k[b, h].T, -np.inf)
+        out[b, h] = np.sum(s == s.max(axis=1, keepdims=True), axis=1)
+    return out
+
+
+def attention_fwd_bf16p(q, k, v, causal: bool, scale: float, fix_mode: int,
+                        round_p: bool = True, return_pbar: bool = False):
+    """Attention with the safe-softmax shift, BF16-rounded P_bar and the fix.
+
+    Per row i (one shift for the whole row):
+      m_i    = max_j S_ij over visible keys,
+      c_i    = #{j : S_ij == m_i}  (exact ties of the raw dot products),
+      m'_i   = m_i + DELTA_NAT if fix_mode == 1 and c_i >= 2, else m_i,
+      P_ij   = exp(S_ij - m'_i),          l_i = sum_j P_ij (unrounded),
+      P_bar  = bf16(P) if round_p else P,
+      O_i    = (sum_j P_bar_ij V_j) / l_i,  LSE_i = m'_i + log l_i.
+    fix_mode 0 leaves the shift at the maximum, so repeated maxima give
+    P_bar == 1 exactly; fix_mode 1 maps them to 1 - 2^-8.
+    """
+    if fix_mode not in (0, 1):
+        raise ValueError("fix_mode must be 0 or 1")
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    o = np.empty((B, H, N, v.shape[-1]))
+    lse = np.empty((B, H, N))
+    pbars = np.empty((B, H, N, N)) if return_pbar else None
+    vis = _mask(N, causal)
+    for b, h in _heads(q):
+        raw = np.where(vis, q[b, h] @ k[b, h].T, -np.inf)
+        ties = np.sum(raw == raw.max(axis=1, keepdims=True), axis=1, keepdims=True)
+        s = scale * raw
+        m = s.max(axis=1, keepdims=True)
+        shift = m + (DELTA_NAT if fix_mode == 1 else 0.0) * (ties >= 2)
+        p = np.exp(s - shift)
+        l = p.sum(axis=1, keepdims=True)
+        pbar = bf16_round(p) if round_p else p
+        o[b, h] = (pbar @ v[b, h]) / l
+        lse[b, h] = shift[:, 0] + np.log(l[:, 0])
+        if return_pbar:
+            pbars[b, h] = pbar
+    if return_pbar:
+        return o, lse, pbars
+    return o, lse

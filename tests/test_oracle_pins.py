@@ -1,0 +1,349 @@
+"""Pins for the FP64 oracle: it is checked against things other than itself.
+
+The pages print no worked example, so the oracle is pinned by
+* brute force: scalar Python loops of the attention definition on tiny inputs
+  ("Is Flash Attention Stable?", the standard-attention definition it measures
+  FlashAttention against);
+* closed forms: equal scores give the (prefix) mean of V, one key gives V_0,
+  a dominant score gives that key's value row;
+* invariants: rows of P sum to one (V = 1 gives O = 1), key permutation
+  equivariance, causal locality, shift invariance of the exact result;
+* finite differences of the brute-force forward for the backward pass;
+* torch's CPU float32 -> bf16 cast for the bf16 rounding;
+* the fix's defining property ("Why Low-Precision Transformer Training Fails",
+  mechanism 2): on repeated-max rows every P_bar, the maxima included, is
+  strictly below 1 (exactly 1 - 2^-8 at the maxima); without it they are 1.
+
+A mutation suite then plants plausible mistakes in a copy of the oracle's
+source and checks that each one trips at least one pin.
+"""
+import math
+import os
+import types
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention64 as ORACLE
+
+ORACLE_SRC = os.path.join(os.path.dirname(ORACLE.__file__), "attention64.py")
+
+
+# ----------------------------------------------------------------------------
+# independent scalar references (pure Python loops, tiny inputs only)
+# ----------------------------------------------------------------------------
+
+def brute_fwd(q, k, v, causal, scale):
+    """Scalar attention of one head: lists in, lists out."""
+    n, d, dv = len(q), len(q[0]), len(v[0])
+    out, lse = [], []
+    for i in range(n):
+        keys = range(i + 1) if causal else range(n)
+        s = [scale * sum(q[i][t] * k[j][t] for t in range(d)) for j in keys]
+        mx = max(s)
+        e = [math.exp(x - mx) for x in s]
+        z = sum(e)
+        out.append([sum(e[a] * v[j][c] for a, j in enumerate(keys)) / z for c in range(dv)])
+        lse.append(mx + math.log(z))
+    return out, lse
+
+
+def brute_ties(q, k, causal):
+    n, d = len(q), len(q[0])
+    res = []
+    for i in range(n):
+        keys = range(i + 1) if causal else range(n)
+        s = [sum(q[i][t] * k[j][t] for t in range(d)) for j in keys]
+        res.append(sum(1 for x in s if x == max(s)))
+    return res
+
+
+def _rand(rng, *shape, scale=1.0):
+    return scale * rng.standard_normal(shape)
+
+
+# ----------------------------------------------------------------------------
+# pin suites: each takes an oracle module and returns the names of failed pins
+# ----------------------------------------------------------------------------
+
+def fwd_pins(M):
+    failed = []
+    rng = np.random.default_rng(1)
+    # P1 brute force, causal and not, odd sizes
+    ok = True
+    for causal in (True, False):
+        q, k, v = _rand(rng, 1, 2, 5, 3), _rand(rng, 1, 2, 5, 3), _rand(rng, 1, 2, 5, 4)
+        o, lse = M.attention_fwd(q, k, v, causal, 0.7)
+        for h in range(2):
+            bo, bl = brute_fwd(q[0, h].tolist(), k[0, h].tolist(), v[0, h].tolist(), causal, 0.7)
+            ok &= np.allclose(o[0, h], bo, rtol=0, atol=1e-12)
+            ok &= np.allclose(lse[0, h], bl, rtol=0, atol=1e-12)
+    if not ok:
+        failed.append("brute_force")
+    # P2 equal scores: Q = 0 -> prefix mean of V and LSE = log(#visible)
+    n = 9
+    q = np.zeros((1, 1, n, 4))
+    k, v = _rand(rng, 1, 1, n, 4), _rand(rng, 1, 1, n, 3)
+    o, lse = M.attention_fwd(q, k, v, True, 0.5)
+    pref = np.cumsum(v[0, 0], axis=0) / np.arange(1, n + 1)[:, None]
+    if not (np.allclose(o[0, 0], pref, atol=1e-13) and np.allclose(lse[0, 0], np.log(np.arange(1, n + 1)), atol=1e-13)):
+        failed.append("equal_scores")
+    o, lse = M.attention_fwd(q, k, v, False, 0.5)
+    if not (np.allclose(o[0, 0], v[0, 0].mean(0), atol=1e-13) and np.allclose(lse[0, 0], math.log(n), atol=1e-13)):
+        failed.append("equal_scores_full")
+    # P3 a single key: O = V_0, LSE = scale * q.k
+    q, k, v = _rand(rng, 1, 1, 1, 5), _rand(rng, 1, 1, 1, 5), _rand(rng, 1, 1, 1, 5)
+    o, lse = M.attention_fwd(q, k, v, True, 0.3)
+    if not (np.allclose(o, v, atol=1e-14) and abs(lse[0, 0, 0] - 0.3 * float(q[0, 0, 0] @ k[0, 0, 0])) < 1e-13):
+        failed.append("single_key")
+    # P4 rows of P sum to one: V = 1 gives O = 1
+    q, k = _rand(rng, 2, 1, 7, 3, scale=3), _rand(rng, 2, 1, 7, 3, scale=3)
+    o, _ = M.attention_fwd(q, k, np.ones((2, 1, 7, 2)), True, 1.0)
+    if not np.allclose(o, 1.0, atol=1e-13):
+        failed.append("rows_sum_to_one")
+    # P5 key permutation equivariance (non-causal): permute K and V rows together
+    q, k, v = _rand(rng, 1, 1, 6, 3), _rand(rng, 1, 1, 6, 3), _rand(rng, 1, 1, 6, 3)
+    perm = rng.permutation(6)
+    o1, l1 = M.attention_fwd(q, k, v, False, 0.9)
+    o2, l2 = M.attention_fwd(q, k[:, :, perm], v[:, :, perm], False, 0.9)
+    if not (np.allclose(o1, o2, atol=1e-13) and np.allclose(l1, l2, atol=1e-13)):
+        failed.append("permutation")
+    # P6 causal locality: rows <= i0 ignore keys/values beyond i0
+    q, k, v = _rand(rng, 1, 1, 8, 3), _rand(rng, 1, 1, 8, 3), _rand(rng, 1, 1, 8, 3)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, 5:] += 10.0
+    v2[:, :, 5:] -= 3.0
+    o1, l1 = M.attention_fwd(q, k, v, True, 1.0)
+    o2, l2 = M.attention_fwd(q, k2, v2, True, 1.0)
+    if not (np.array_equal(o1[:, :, :5], o2[:, :, :5]) and np.array_equal(l1[:, :, :5], l2[:, :, :5])
+            and not np.allclose(o1[:, :, 5:], o2[:, :, 5:])):
+        failed.append("causal_locality")
+    # P7 a dominant score: S_ij* = G above every other score pulls O_i to V_j*
+    n, G = 6, 30.0
+    k = _rand(rng, 1, 1, n, 4, scale=1e-3)
+    q = np.zeros((1, 1, n, 4))
+    q[0, 0, :, 0] = G
+    k[0, 0, 2, 0] = 1.0
+    v = _rand(rng, 1, 1, n, 3)
+    o, _ = M.attention_fwd(q, k, v, False, 1.0)
+    bound = (n - 1) * math.exp(-(G - 2 * G * 1e-3 * 4)) * 2 * np.abs(v).max()
+    if not np.all(np.abs(o[0, 0] - v[0, 0, 2]) <= bound):
+        failed.append("dominant_score")
+    return failed
+
+
+def bwd_pins(M):
+    """Central finite differences of the brute-force forward, L = sum(dO * O)."""
+    failed = []
+    rng = np.random.default_rng(2)
+    for causal in (True, False):
+        q, k, v = _rand(rng, 1, 1, 4, 3), _rand(rng, 1, 1, 4, 3), _rand(rng, 1, 1, 4, 2)
+        do = _rand(rng, 1, 1, 4, 2)
+        scale = 0.8
+        dq, dk, dv = M.attention_bwd(q, k, v, do, causal, scale)
+
+        def loss(qq, kk, vv):
+            o, _ = brute_fwd(qq[0, 0].tolist(), kk[0, 0].tolist(), vv[0, 0].tolist(), causal, scale)
+            return float(np.sum(np.asarray(o) * do[0, 0]))
+
+        h = 1e-6
+        for name, x, g in (("dq", q, dq), ("dk", k, dk), ("dv", v, dv)):
+            fd = np.zeros_like(x)
+            for idx in np.ndindex(*x.shape):
+                xp, xm = x.copy(), x.copy()
+                xp[idx] += h
+                xm[idx] -= h
+                args_p = {"dq": (xp, k, v), "dk": (q, xp, v), "dv": (q, k, xp)}[name]
+                args_m = {"dq": (xm, k, v), "dk": (q, xm, v), "dv": (q, k, xm)}[name]
+                fd[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            if not np.allclose(g, fd, rtol=1e-6, atol=1e-8):
+                failed.append(f"fd_{name}_{'causal' if causal else 'full'}")
+    return failed
+
+
+def bf16_pins(M):
+    failed = []
+    rng = np.random.default_rng(3)
+    x = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32),
+        (rng.standard_normal(20000) * 1e-38).astype(np.float32),   # subnormal range of bf16
+        (rng.standard_normal(5000) * 1e37).astype(np.float32),
+        np.exp(rng.uniform(-30, 0, 20000)).astype(np.float32),      # the range of softmax weights
+    ])
+    edges = np.array([0.0, -0.0, 1.0, 1 + 2 ** -8, 1 + 3 * 2 ** -8, 1 - 2 ** -9, 1 - 3 * 2 ** -9,
+                      0.99609375, 2.0 ** -126, 2.0 ** -133, 2.0 ** -134, 3 * 2.0 ** -135, 2.0 ** -149,
+                      3.3895313892515355e38, 3.3961e38, 3.4e38, np.inf, -np.inf], dtype=np.float32)
+    x = np.concatenate([x, edges, -edges])
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    got = M.bf16_round(x.astype(np.float64))
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    signs = np.signbit(got) == np.signbit(ref)
+    if not (same.all() and signs.all()):
+        failed.append("torch_cast")
+    nan = M.bf16_round(np.array([np.nan]))
+    if not np.isnan(nan).all():
+        failed.append("nan")
+    return failed
+
+
+def _tie_inputs(rng, n=8, d=3):
+    """Small integer-valued inputs with duplicated keys: exact ties by construction."""
+    q = rng.integers(-2, 3, size=(1, 2, n, d)).astype(np.float64)
+    k = rng.integers(-2, 3, size=(1, 2, n, d)).astype(np.float64)
+    v = rng.standard_normal((1, 2, n, 4))
+    k[0, 0, 5] = k[0, 0, 1]
+    k[0, 1, 6] = k[0, 1, 0]
+    return q, k, v
+
+
+def emulation_pins(M):
+    failed = []
+    rng = np.random.default_rng(4)
+    # E1 without rounding the emulation is the exact definition, whatever the fix does
+    q, k, v = _rand(rng, 1, 2, 9, 4), _rand(rng, 1, 2, 9, 4), _rand(rng, 1, 2, 9, 4)
+    k[0, 0, 7] = k[0, 0, 2]
+    o, lse = M.attention_fwd(q, k, v, True, 0.6)
+    for fix in (0, 1):
+        oe, le = M.attention_fwd_bf16p(q, k, v, True, 0.6, fix, round_p=False)
+        if not (np.allclose(oe, o, atol=1e-13) and np.allclose(le, lse, atol=1e-13)):
+            failed.append(f"unrounded_equals_exact_fix{fix}")
+    # E2 the fix's defining property on repeated-max rows
+    q, k, v = _tie_inputs(rng)
+    ties = np.asarray(brute_ties(q[0, 0].tolist(), k[0, 0].tolist(), True))
+    ties1 = np.asarray(brute_ties(q[0, 1].tolist(), k[0, 1].tolist(), True))
+    all_ties = np.stack([ties, ties1])
+    _, _, p0 = M.attention_fwd_bf16p(q, k, v, True, 0.5, 0, return_pbar=True)
+    _, _, p1 = M.attention_fwd_bf16p(q, k, v, True, 0.5, 1, return_pbar=True)
+    rep = all_ties >= 2
+    if not rep.any():
+        failed.append("no_repeated_rows_in_fixture")
+    ok = True
+    for h in range(2):
+        for i in range(q.shape[2]):
+            row0, row1 = p0[0, h, i, : i + 1], p1[0, h, i, : i + 1]
+            if rep[h, i]:
+                ok &= row0.max() == 1.0 and np.sum(row0 == 1.0) == all_ties[h, i]
+                ok &= row1.max() == 1.0 - 2.0 ** -8 and np.all(row1 < 1.0)
+                ok &= np.sum(row1 == 1.0 - 2.0 ** -8) == all_ties[h, i]
+            else:
+                ok &= np.array_equal(row0, row1) and row0.max() == 1.0
+    if not ok:
+        failed.append("fix_property")
+    # E3 rounding P to bf16 moves O by at most 2^-8 * max|V| (unit roundoff of bf16)
+    q, k, v = _rand(rng, 2, 2, 16, 8), _rand(rng, 2, 2, 16, 8), _rand(rng, 2, 2, 16, 8)
+    o, lse = M.attention_fwd(q, k, v, True, 0.35)
+    for fix in (0, 1):
+        oe, le = M.attention_fwd_bf16p(q, k, v, True, 0.35, fix)
+        bound = 2.0 ** -8 * np.abs(v).max(axis=2, keepdims=True)
+        if not (np.all(np.abs(oe - o) <= bound) and np.allclose(le, lse, atol=1e-13)):
+            failed.append(f"rounding_bound_fix{fix}")
+        if np.abs(oe - o).max() < 1e-6:
+            failed.append(f"rounding_not_applied_fix{fix}")
+    # P_bar lies on the bf16 grid (checked with torch's cast, not the oracle's)
+    _, _, pb = M.attention_fwd_bf16p(q, k, v, True, 0.35, 1, return_pbar=True)
+    pb32 = pb.astype(np.float32)
+    if not (np.array_equal(pb32.astype(np.float64), pb) and
+            np.array_equal(torch.from_numpy(pb32).to(torch.bfloat16).float().numpy(), pb32)):
+        failed.append("pbar_off_bf16_grid")
+    # E4 exact tie counts against brute force
+    q, k, v = _tie_inputs(rng)
+    for causal in (True, False):
+        got = M.tie_counts(q, k, causal)
+        exp = np.stack([brute_ties(q[0, h].tolist(), k[0, h].tolist(), causal) for h in range(2)])
+        if not np.array_equal(got[0], exp):
+            failed.append(f"tie_counts_{'causal' if causal else 'full'}")
+    return failed
+
+
+# ----------------------------------------------------------------------------
+# the oracle passes every pin
+# ----------------------------------------------------------------------------
+
+def test_forward_pins():
+    assert fwd_pins(ORACLE) == []
+
+
+def test_backward_pins_finite_differences():
+    assert bwd_pins(ORACLE) == []
+
+
+def test_bf16_rounding_matches_torch_cast():
+    assert bf16_pins(ORACLE) == []
+
+
+def test_emulation_and_fix_pins():
+    assert emulation_pins(ORACLE) == []
+
+
+def test_delta_constant():
+    # the shift maps a maximum to exactly the largest bf16 value below 1
+    assert ORACLE.bf16_round(np.exp(-ORACLE.DELTA_NAT)) == 0.99609375
+    assert ORACLE.bf16_round(2.0 ** -ORACLE.DELTA_LOG2) == 0.99609375
+    assert abs(ORACLE.DELTA_NAT - ORACLE.DELTA_LOG2 * math.log(2)) < 1e-16
+
+
+def test_hand_worked_example():
+    """tests/golden/handworked_2x2.txt: two keys whose scores differ by ln 3."""
+    path = os.path.join(os.path.dirname(__file__), "golden", "handworked_2x2.txt")
+    vals = {}
+    for line in open(path):
+        line = line.split("#", 1)[0].strip()
+        if line:
+            key, rhs = line.split("=", 1)
+            vals[key.strip()] = np.array([float(eval(t, {"ln": math.log, "sqrt": math.sqrt}))
+                                          for t in rhs.split()])
+    q = vals["q"].reshape(1, 1, 1, 2)
+    k = vals["k"].reshape(1, 1, 2, 2)
+    v = vals["v"].reshape(1, 1, 2, 2)
+    # one query against two keys, non-causal
+    o, lse = ORACLE.attention_fwd(np.repeat(q, 2, axis=2), k, v, False, float(vals["scale"][0]))
+    assert np.allclose(o[0, 0, 0], vals["o"], atol=1e-15)
+    assert abs(lse[0, 0, 0] - vals["lse"][0]) < 1e-15
+
+
+# ----------------------------------------------------------------------------
+# planted mistakes: each must trip at least one pin
+# ----------------------------------------------------------------------------
+
+MUTATIONS = [
+    ("fwd_drops_scale", "s = scale * (q[b, h] @ k[b, h].T)\n        s = np.where(vis, s, -np.inf)\n        m = s.max(axis=1, keepdims=True)\n        e = np.exp(s - m)\n        l = e",
+     "s = (q[b, h] @ k[b, h].T)\n        s = np.where(vis, s, -np.inf)\n        m = s.max(axis=1, keepdims=True)\n        e = np.exp(s - m)\n        l = e"),
+    ("fwd_wrong_operand", "o[b, h] = p @ v[b, h]\n        lse", "o[b, h] = p @ k[b, h][:, : v.shape[-1]]\n        lse"),
+    ("mask_off_by_one", "np.tril(np.ones((n, n), dtype=bool))", "np.tril(np.ones((n, n), dtype=bool), k=1)"),
+    ("lse_drops_max", "lse[b, h] = m[:, 0] + np.log(l[:, 0])", "lse[b, h] = np.log(l[:, 0])"),
+    ("dv_not_transposed", "dv[b, h] = p.T @ do[b, h]", "dv[b, h] = p @ do[b, h]"),
+    ("ds_drops_D", "ds = p * (dp - D)", "ds = p * dp"),
+    ("ds_wrong_sign", "ds = p * (dp - D)", "ds = p * (D - dp)"),
+    ("dk_not_transposed", "dk[b, h] = scale * (ds.T @ q[b, h])", "dk[b, h] = scale * (ds @ q[b, h])"),
+    ("dq_drops_scale", "dq[b, h] = scale * (ds @ k[b, h])", "dq[b, h] = (ds @ k[b, h])"),
+    ("bf16_one_bit_short", "q_exp = np.maximum(e, -125) - 8", "q_exp = np.maximum(e, -125) - 7"),
+    ("bf16_truncates", "np.rint(np.ldexp(xf, -q_exp))", "np.trunc(np.ldexp(xf, -q_exp))"),
+    ("bf16_no_subnormals", "q_exp = np.maximum(e, -125) - 8", "q_exp = e - 8"),
+    ("fix_on_every_row", "* (ties >= 2)", "* (ties >= 1)"),
+    ("fix_wrong_delta", "DELTA_NAT = -np.log(1.0 - 2.0 ** -8)", "DELTA_NAT = -np.log(1.0 - 2.0 ** -6)"),
+    ("emulation_skips_rounding", "pbar = bf16_round(p) if round_p else p", "pbar = p"),
+    ("ties_ignore_mask", "s = np.where(vis, q[b, h] @ k[b, h].T, -np.inf)\n        out[b, h]", "s = q[b, h] @ k[b, h].T\n        out[b, h]"),
+]
+
+
+def _mutant(old, new):
+    src = open(ORACLE_SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique: {old!r}"
+    mod = types.ModuleType("oracle_mutant")
+    exec(compile(src.replace(old, new), "oracle_mutant", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(name, old, new):
+    M = _mutant(old, new)
+    failed = []
+    for suite in (fwd_pins, bf16_pins, emulation_pins, bwd_pins):
+        try:
+            failed += suite(M)
+        except Exception as exc:  # a mutant that cannot even run fails its pins
+            failed.append(f"{suite.__name__}: {type(exc).__name__}")
+        if failed:
+            break
+    assert failed, f"mutation {name} passed every pin"
