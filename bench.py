@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark: BF16 attention forward + backward on B200, repeated-max fix on.
+
+One step = fa_fwd + fa_bwd (the whole hot path) over one batch of synthetic
+input of the chosen workload (default: GPT-2 small attention, B=8 H=12 N=1024
+d=64, causal).  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the FP64 CPU oracle, timed on host cores
+
+Timing: CUDA events on the launching stream around every launch of every
+step; the L2 is flushed (a 512 MiB write) before each step, outside the
+events.  Multi-GPU runs are independent replicas (attention over (B, H) has no
+exchange step): each rank runs the full workload on its own GPU, and the
+slowest rank's time is used.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from flashattention_bf16_fwd_b200.workloads import WORKLOADS, make_inputs, visible_pairs, workload_flops  # noqa: E402
+
+METRIC = "BF16 attn fwd+bwd TFLOP/s (% of B200 BF16 peak), fix on; max err vs FP64 oracle"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_BF16_TFLOPS = 2250.0
+L2_FLUSH_BYTES = 512 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt2s")
+    ap.add_argument("--fix-mode", type=int, default=1)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def all_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU is busy."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def mark(self, begin: bool):
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        busy = [s for s, r in zip(sm, rows) if float(r[3]) > 150.0] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median(busy)), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows)}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(x, w, budget_s, seed=0, gpu_out=None):
+    """Time the FP64 oracle (forward + backward) on seeded heads until the budget is spent.
+
+    Returns (algorithmic FLOPs done, seconds, heads, errors vs the GPU outputs of the same heads).
+    """
+    from flashattention_bf16_fwd_b200.stats import lse_rel_err, max_rel_err, normwise_rel_err
+    from oracle import attention_bwd, attention_fwd
+
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(w.B * w.H)
+    per_head = workload_flops(1, 1, w.N, w.d, w.causal)["total"]
+    flops = secs = 0.0
+    heads = []
+    errs = {"o_max_abs": 0.0, "o_max_rel": 0.0, "lse_rel": 0.0, "dq_rel": 0.0, "dk_rel": 0.0, "dv_rel": 0.0}
+    for idx in order:
+        b, h = divmod(int(idx), w.H)
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        xs = {n: x[n][sl] for n in ("q", "k", "v", "do")}
+        t0 = time.perf_counter()
+        o_ref, lse_ref = attention_fwd(xs["q"], xs["k"], xs["v"], w.causal, w.scale)
+        grads = attention_bwd(xs["q"], xs["k"], xs["v"], xs["do"], w.causal, w.scale)
+        secs += time.perf_counter() - t0
+        flops += per_head
+        heads.append((b, h))
+        if gpu_out is not None:
+            g = {n: t[sl].float().cpu().numpy() for n, t in gpu_out.items()}
+            errs["o_max_abs"] = max(errs["o_max_abs"], float(np.abs(g["o"] - o_ref).max()))
+            errs["o_max_rel"] = max(errs["o_max_rel"], max_rel_err(g["o"], o_ref))
+            errs["lse_rel"] = max(errs["lse_rel"], lse_rel_err(g["lse"], lse_ref))
+            for n, r in zip(("dq", "dk", "dv"), grads):
+                errs[f"{n}_rel"] = max(errs[f"{n}_rel"], normwise_rel_err(g[n], r))
+        if secs >= budget_s:
+            break
+    return flops, secs, heads, (errs if gpu_out is not None else None)
+
+
+def run_reference(args, rank, world):
+    """The FP64 CPU oracle as the reference arm, on bounded samples of the workload."""
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w, seed=args.seed)
+    per_step_budget = max(0.5, 60.0 / max(args.steps + args.warmup, 1))
+    for _ in range(args.warmup):
+        oracle_sample(x, w, per_step_budget / 4, seed=args.seed)
+    flops = secs = 0.0
+    heads = 0
+    for i in range(args.steps):
+        f, s, hs, _ = oracle_sample(x, w, per_step_budget, seed=args.seed + 1 + i)
+        flops, secs, heads = flops + f, secs + s, heads + len(hs)
+    value = flops / secs / 1e12
+    cores = cpu_threads()
+    sample = (f"{heads} (batch, head) pairs of {args.workload} over {args.steps} steps, "
+              f"fwd+bwd FP64 NumPy oracle, ~{per_step_budget:.1f} s per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, args),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, args):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} {'causal' if w.causal else 'full'}, "
+                        f"{w.structure} inputs, fix_mode={args.fix_mode}",
+            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "fix_mode": args.fix_mode,
+            "parallelism": "replicas", "l2": "flushed before every step (512 MiB write, outside the events)"}
+
+
+def run_ours(args, rank, world, local):
+    from flashattention_bf16_fwd_b200 import fa
+
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local if world > 1 else 0)
+    x = make_inputs(w, seed=args.seed + rank)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.fa_bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    causal, scale, fix = w.causal, w.scale, args.fix_mode
+
+    def check(rc, what):
+        if rc != 0:
+            raise RuntimeError(f"{what}: {fa.fa_status_string(rc)}")
+
+    def step(ev):
+        ev[0].record(stream)
+        check(fa.fa_fwd(q, k, v, o, lse, causal, scale, fix, stream), "fa_fwd")
+        ev[1].record(stream)
+        check(fa.fa_bwd_preprocess(o, do, ws, stream), "fa_bwd_preprocess")
+        ev[2].record(stream)
+        check(fa.fa_bwd_main(q, k, v, lse, do, dk, dv, ws, causal, scale, stream), "fa_bwd_main")
+        ev[3].record(stream)
+        check(fa.fa_bwd_finish(dq, ws, scale, stream), "fa_bwd_finish")
+        ev[4].record(stream)
+
+    launches_per_step = 4
+    warm = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step(warm)
+    torch.cuda.synchronize()
+    check(fa.fa_check_device_error(), "warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    sampler = ClockSampler(local if world > 1 else 0)
+    sampler.start()
+    time.sleep(0.2)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.mark(True)
+    outer[0].record(stream)
+    for i in range(args.steps):
+        flush.zero_()
+        step(events[i])
+    outer[1].record(stream)
+    torch.cuda.synchronize()
+    sampler.mark(False)
+    barrier(world)
+    clocks = sampler.stop()
+    check(fa.fa_check_device_error(), "timed steps")
+
+    per = np.array([[events[i][j].elapsed_time(events[i][j + 1]) for j in range(4)] for i in range(args.steps)])
+    step_ms = per.sum(axis=1)
+    t_rank = float(step_ms.sum())
+    t_max = all_max(t_rank, world)
+    outer_ms = all_max(outer[0].elapsed_time(outer[1]), world)
+    flops = workload_flops(w.B, w.H, w.N, w.d, w.causal)
+    value = world * args.steps * flops["total"] / (t_max * 1e-3) / 1e12
+
+    peaks, peak_kind = load_peaks()
+    kern_names = ["fa_fwd_kernel", "fa_bwd_pre_kernel", "fa_bwd_kernel", "fa_bwd_dq_kernel"]
+    kern_ms = per.mean(axis=0)
+    rows = w.B * w.H * w.N
+    elem = rows * w.d
+    work = {
+        "fa_fwd_kernel": ("tensor", flops["fwd"]),
+        "fa_bwd_pre_kernel": ("hbm", 2 * elem * 2 + rows * 4 + elem * 4),
+        "fa_bwd_kernel": ("tensor", flops["bwd"]),
+        "fa_bwd_dq_kernel": ("hbm", elem * 4 + elem * 2),
+    }
+    kernels = {}
+    for name, ms in zip(kern_names, kern_ms):
+        bound, amount = work[name]
+        rate = amount / (ms * 1e-3)
+        kernels[name] = {"ms": float(ms), "share": float(ms / kern_ms.sum()),
+                         ("TFLOP/s" if bound == "tensor" else "GB/s"): rate / (1e12 if bound == "tensor" else 1e9)}
+    dom = kern_names[int(np.argmax(kern_ms))]
+    bound, amount = work[dom]
+    if bound == "tensor":
+        achieved, peak, unit = amount / (kern_ms[kern_names.index(dom)] * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    else:
+        achieved, peak, unit = amount / (kern_ms[kern_names.index(dom)] * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
+    traffic = measured_traffic(dom, w)
+    roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_kind} burst",
+                "algorithmic": amount}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(fa, x, w, args, dev, stream, flops["total"], world)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w, args),
+        "pct_of_peak": {"measured_burst": value / world / peaks["bf16_tflops"] * 100.0,
+                        "datasheet": value / world / DATASHEET_BF16_TFLOPS * 100.0, "peak_source": peak_kind},
+        "ms_per_step_bracket": outer_ms / args.steps,
+        "roofline": roofline, "kernels": kernels, "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gout = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+        fl, secs, heads, errs = oracle_sample(x, w, args.cpu_seconds, seed=args.seed, gpu_out=gout)
+        line["cpu_baseline"] = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
+                                "kind": "oracle",
+                                "sample": f"{len(heads)} of {w.B * w.H} (batch, head) pairs, FP64 NumPy "
+                                          f"fwd+bwd, {secs:.1f} s; errors measured on the same heads"}
+        line["max_err"] = errs
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def measured_traffic(kernel, w):
+    """DRAM bytes per launch from the committed ncu capture, if it matches this kernel build."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    import hashlib
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "flashattention_bf16_fwd_b200", "csrc")
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(src)):
+        with open(os.path.join(src, fn), "rb") as f:
+            h.update(f.read())
+    if rec.get("csrc_sha256") != h.hexdigest():
+        return None
+    if rec.get("workload") != w.name:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def run_e2e(fa, x, w, args, dev, stream, flops_total, world):
+    """Same metric end to end: pinned host inputs -> device -> fa_fwd + fa_bwd -> host outputs, every step."""
+    host_in = {n: x[n].pin_memory() for n in ("q", "k", "v", "do")}
+    dev_in = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
+    shape = (w.B, w.H, w.N, w.d)
+    host_out = {n: torch.empty(shape, dtype=torch.bfloat16).pin_memory() for n in ("o", "dq", "dk", "dv")}
+    host_out["lse"] = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+    dev_out = {n: torch.empty_like(t, device=dev) for n, t in host_out.items()}
+    ws = torch.empty(fa.fa_bwd_workspace_size(*shape), dtype=torch.uint8, device=dev)
+
+    def one():
+        for n in host_in:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        rc = fa.fa_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_out["o"], dev_out["lse"], w.causal, w.scale,
+                       args.fix_mode, stream)
+        rc |= fa.fa_bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_out["o"], dev_out["lse"], dev_in["do"],
+                        dev_out["dq"], dev_out["dk"], dev_out["dv"], ws, w.causal, w.scale, stream)
+        if rc != 0:
+            raise RuntimeError("e2e step failed")
+        for n in host_out:
+            host_out[n].copy_(dev_out[n], non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 20))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier(world)
+    ev[0].record(stream)
+    for _ in range(steps):
+        one()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    t = all_max(ev[0].elapsed_time(ev[1]), world)
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    return {"value": world * steps * flops_total / (t * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": t / steps}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores only; other ranks have no work
+        run_reference(args, int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")))
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

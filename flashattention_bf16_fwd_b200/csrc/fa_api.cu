@@ -1,0 +1,292 @@
+// fa_api.cu - the C ABI declared in include/fa_b200.h: argument checks, TMA
+// tensor maps, launch configuration, and the device error flag.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/fa_b200.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace fa {
+
+// Set by a kernel whose bounded wait expired; read and cleared by
+// fa_check_device_error().
+__device__ int g_dev_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  std::once_flag once;
+  int ok = 0;            // 1 when the device is sm_100 and the flag address is known
+  int num_sms = 0;
+  int* dev_error = nullptr;
+};
+DeviceState g_devices[kMaxDevices];
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// Per-device set-up, done once with that device current: check the
+// architecture, opt the kernels into large shared memory, and resolve the
+// device address of the error flag.
+DeviceState* device_state() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  DeviceState* st = &g_devices[dev];
+  std::call_once(st->once, [st, dev] {
+    cudaDeviceProp prop{};
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess || prop.major != 10) return;
+    st->num_sms = prop.multiProcessorCount;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_dev_error) != cudaSuccess) return;
+    st->dev_error = static_cast<int*>(addr);
+    bool ok = true;
+    ok &= cudaFuncSetAttribute(fa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdLayout<64>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdLayout<128>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(fa_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdLayout<64>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(fa_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdLayout<128>::kAlloc) == cudaSuccess;
+    st->ok = ok ? 1 : 0;
+  });
+  return st->ok ? st : nullptr;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int H, int N, int d, int causal, float scale) {
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
+  const long long total = (long long)B * H * N * d;
+  if (total >= (1ll << 31)) return FA_ERR_SHAPE;
+  if (causal != 0 && causal != 1) return FA_ERR_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_ARG;
+  return FA_OK;
+}
+
+// A [BH, N, D] bf16 tensor seen as 3-D (d, n, bh); boxes of 64 x 128 x 1 with
+// the 128-byte swizzle the tcgen05 descriptors expect.  Rows past N read 0.
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(N), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(N) * D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Shift added to m on repeated-max rows (base-2 units): maps a maximum to 1 - 2^-8.
+const double kDeltaLog2 = -std::log2(1.0 - 1.0 / 256.0);
+
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties, int B, int H,
+               int N, int d, int causal, float scale, int fix_mode, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  int rc = check_common(B, H, N, d, causal, scale);
+  if (rc != FA_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGN;
+  if (fix_mode != 0 && fix_mode != 1) return FA_ERR_FIXMODE;
+  DeviceState* st = device_state();
+  if (!st) return FA_ERR_DEVICE;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, BH, N, d) || !make_map(&mk, k, BH, N, d) || !make_map(&mv, v, BH, N, d))
+    return FA_ERR_DEVICE;
+  FwdParams prm{};
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.ties = ties;
+  prm.dev_error = st->dev_error;
+  prm.BH = BH;
+  prm.N = N;
+  prm.n_pairs = (N + 255) / 256;
+  prm.causal = causal;
+  prm.scale_log2 = float(double(scale) * 1.4426950408889634);
+  prm.delta_log2 = fix_mode ? float(kDeltaLog2) : 0.f;
+  prm.fix = fix_mode;
+  const dim3 grid(unsigned(prm.n_pairs) * unsigned(BH));
+  if (d == 64)
+    fa_fwd_kernel<64><<<grid, FwdLayout<64>::kThreads, FwdLayout<64>::kAlloc, stream>>>(mq, mk, mv, prm);
+  else
+    fa_fwd_kernel<128><<<grid, FwdLayout<128>::kThreads, FwdLayout<128>::kAlloc, stream>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           int causal, float scale, int fix_mode, void* stream) {
+  return launch_fwd(q, k, v, o, lse, nullptr, B, H, N, d, causal, scale, fix_mode,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_ties(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties, int B, int H,
+                int N, int d, int causal, float scale, int fix_mode, void* stream) {
+  if (!ties) return FA_ERR_NULL;
+  return launch_fwd(q, k, v, o, lse, ties, B, H, N, d, causal, scale, fix_mode,
+                    static_cast<cudaStream_t>(stream));
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_common(B, H, N, d, 0, 1.f) != FA_OK) return 0;
+  const size_t rows = size_t(B) * H * N;
+  return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+int fa_bwd_preprocess(const void* o, const void* dout, void* workspace, size_t workspace_bytes, int B, int H,
+                      int N, int d, void* stream) {
+  if (!o || !dout) return FA_ERR_NULL;
+  int rc = check_common(B, H, N, d, 0, 1.f);
+  if (rc != FA_OK) return rc;
+  if (!aligned16(o) || !aligned16(dout)) return FA_ERR_ALIGN;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, N, d))
+    return FA_ERR_WORKSPACE;
+  if (!device_state()) return FA_ERR_DEVICE;
+  const size_t rows = size_t(B) * H * N;
+  float* dq_acc = static_cast<float*>(workspace);
+  float* dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256(rows * d * sizeof(float)));
+  const int threads = 256;
+  const long long blocks = ((long long)rows * 8 + threads - 1) / threads;
+  fa_bwd_pre_kernel<<<unsigned(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), dsum, dq_acc,
+      (long long)rows, d);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dout, void* dk,
+                void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d, int causal,
+                float scale, void* stream) {
+  if (!q || !k || !v || !lse || !dout || !dk || !dv) return FA_ERR_NULL;
+  int rc = check_common(B, H, N, d, causal, scale);
+  if (rc != FA_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_ALIGN;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, N, d))
+    return FA_ERR_WORKSPACE;
+  DeviceState* st = device_state();
+  if (!st) return FA_ERR_DEVICE;
+  const int BH = B * H;
+  const size_t rows = size_t(BH) * N;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, q, BH, N, d) || !make_map(&mk, k, BH, N, d) || !make_map(&mv, v, BH, N, d) ||
+      !make_map(&mdo, dout, BH, N, d))
+    return FA_ERR_DEVICE;
+  BwdParams prm{};
+  prm.lse = lse;
+  prm.dsum = reinterpret_cast<const float*>(static_cast<uint8_t*>(workspace) + align256(rows * d * sizeof(float)));
+  prm.dq_acc = static_cast<float*>(workspace);
+  prm.dk = static_cast<__nv_bfloat16*>(dk);
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.dev_error = st->dev_error;
+  prm.BH = BH;
+  prm.N = N;
+  prm.n_kv = (N + 127) / 128;
+  prm.causal = causal;
+  prm.scale = scale;
+  prm.scale_log2 = float(double(scale) * 1.4426950408889634);
+  const dim3 grid(unsigned(prm.n_kv) * unsigned(BH));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    fa_bwd_kernel<64><<<grid, BwdLayout<64>::kThreads, BwdLayout<64>::kAlloc, s>>>(mq, mk, mv, mdo, prm);
+  else
+    fa_bwd_kernel<128><<<grid, BwdLayout<128>::kThreads, BwdLayout<128>::kAlloc, s>>>(mq, mk, mv, mdo, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+int fa_bwd_finish(void* dq, const void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale,
+                  void* stream) {
+  if (!dq) return FA_ERR_NULL;
+  int rc = check_common(B, H, N, d, 0, scale);
+  if (rc != FA_OK) return rc;
+  if (!aligned16(dq)) return FA_ERR_ALIGN;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, N, d))
+    return FA_ERR_WORKSPACE;
+  if (!device_state()) return FA_ERR_DEVICE;
+  const long long n8 = (long long)B * H * N * d / 8;
+  const int threads = 256;
+  fa_bwd_dq_kernel<<<unsigned((n8 + threads - 1) / threads), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const float*>(workspace), static_cast<__nv_bfloat16*>(dq), scale, n8);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+           void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+           int causal, float scale, void* stream) {
+  // Check everything up front so that an error leaves every output untouched.
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
+  int rc = check_common(B, H, N, d, causal, scale);
+  if (rc != FA_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_ALIGN;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, N, d))
+    return FA_ERR_WORKSPACE;
+  if (!device_state()) return FA_ERR_DEVICE;
+  rc = fa_bwd_preprocess(o, dout, workspace, workspace_bytes, B, H, N, d, stream);
+  if (rc != FA_OK) return rc;
+  rc = fa_bwd_main(q, k, v, lse, dout, dk, dv, workspace, workspace_bytes, B, H, N, d, causal, scale, stream);
+  if (rc != FA_OK) return rc;
+  return fa_bwd_finish(dq, workspace, workspace_bytes, B, H, N, d, scale, stream);
+}
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_NULL: return "a required pointer is NULL";
+    case FA_ERR_SHAPE: return "B, H or N < 1, or B*H*N*d >= 2^31";
+    case FA_ERR_HEADDIM: return "head dimension d must be 64 or 128";
+    case FA_ERR_ALIGN: return "a tensor base address is not 16-byte aligned";
+    case FA_ERR_FIXMODE: return "fix_mode must be 0 or 1";
+    case FA_ERR_WORKSPACE: return "workspace is NULL, misaligned or smaller than fa_bwd_workspace_size()";
+    case FA_ERR_LAUNCH: return "the CUDA runtime refused a kernel launch";
+    case FA_ERR_TIMEOUT: return "a kernel gave up on a bounded wait (device error flag set)";
+    case FA_ERR_ARG: return "causal must be 0 or 1 and scale finite and > 0";
+    case FA_ERR_DEVICE: return "no sm_100 device, or tensor-map encoding unavailable";
+    default: return "unknown status";
+  }
+}
+
+int fa_check_device_error(void* stream) {
+  DeviceState* st = device_state();
+  if (!st) return FA_ERR_DEVICE;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
+  int flag = 0;
+  if (cudaMemcpy(&flag, st->dev_error, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_LAUNCH;
+  if (flag != kDevErrNone) {
+    const int zero = 0;
+    cudaMemcpy(st->dev_error, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    return flag == kDevErrTimeout ? FA_ERR_TIMEOUT : FA_ERR_DEVICE;
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,334 @@
+// fa_fwd.cuh - forward pass: tiled attention with an online safe softmax, the
+// repeated-max fix, a BF16 rounding point for P_bar, and the log-sum-exp.
+//
+// Method: "Is Flash Attention Stable?" (chibakuma.com) describes the tiling:
+// Q/K/V are cut into blocks held on chip, each block is scaled and folded into
+// a running result, so the N x N score matrix never reaches HBM.  "Why
+// Low-Precision Transformer Training Fails" (admirer.cn summary, mechanism 2)
+// places the bias in the unnormalised output P_bar V and gives the fix: when
+// the row maximum of S occurs more than once, raise the shift m so every
+// exponent, the maxima included, is strictly below 1.
+//
+// One CTA = one (batch, head) and two 128-row query tiles, processed in
+// ping-pong so the tensor core works on one tile while the other tile's
+// softmax runs on the CUDA cores:
+//   warps 0-3  softmax of query tile 0 (thread r owns row r: TMEM lane r)
+//   warps 4-7  softmax of query tile 1
+//   warp  8    TMA producer: Q tiles once, then a ring of K/V stages
+//   warp  9    TMEM allocator + single-thread tcgen05.mma issuer
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 after.
+// P_bar (bf16, two per 32-bit column) overwrites the first 64 columns of S_t
+// and is the A operand of O_t += P_bar V (V is the MN-major B operand).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  __nv_bfloat16* o;     // [BH, N, D]
+  float* lse;           // [BH, N]
+  int32_t* ties;        // [BH, N] or nullptr
+  int* dev_error;       // library error flag
+  int BH, N, n_pairs, causal;
+  float scale_log2;     // scale * log2(e): S -> base-2 exponent domain
+  float delta_log2;     // shift added to m on repeated-max rows (0 = fix off)
+  int fix;
+};
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kStages = (D == 64) ? 4 : 2;   // K/V ring depth
+  static constexpr int kSub = D / 64;                 // 64-column sub-tiles per 128-row tile
+  static constexpr int kSubBytes = 128 * 64 * 2;      // one TMA box, 16 KB
+  static constexpr int kTileBytes = kSub * kSubBytes; // a 128 x D bf16 tile
+  static constexpr int kQOff = 0;                     // Q0, Q1
+  static constexpr int kKVOff = 2 * kTileBytes;       // stage s: K, then V
+  static constexpr int kBarOff = kKVOff + kStages * 2 * kTileBytes;
+  static constexpr int kBytes = kBarOff + 256;
+  static constexpr int kAlloc = kBytes + 1024;        // room to align the base to 1 KB
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kThreads = 320;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdLayout<D>;
+  const float kNegInf = -__int_as_float(0x7f800000);
+  constexpr float kLn2 = 0.69314718055994531f;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + L::kStages;
+  uint64_t* s_full = kv_empty + L::kStages;  // [2]
+  uint64_t* p_full = s_full + 2;             // [2]
+  uint64_t* o_done = p_full + 2;             // [2]
+  uint64_t* mma_done = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  // Causal tiles get heavier with the query index: launch the heavy ones first.
+  const int pair = p.causal ? (p.n_pairs - 1 - int(blockIdx.x) / p.BH) : int(blockIdx.x) / p.BH;
+  const int bh = int(blockIdx.x) % p.BH;
+  const int q0_row = pair * 256;
+  const int q1_row = q0_row + 128;
+  const int n_kv = (p.N + 127) / 128;
+  const int n0 = p.causal ? min(2 * pair + 1, n_kv) : n_kv;
+  const int n1 = (q1_row < p.N) ? (p.causal ? min(2 * pair + 2, n_kv) : n_kv) : 0;
+  const int nmax = max(n0, n1);
+
+  const int warp = int(warp_id());
+  const int lane = int(lane_id());
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_done[t], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{abort_flag, p.dev_error};
+
+  if (warp == 8) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint64_t pol_q = l2_policy_evict_first();
+      const uint64_t pol_kv = l2_policy_evict_last();
+      const int nq = (n1 > 0) ? 2 : 1;
+      mbar_arrive_expect_tx(q_full, uint32_t(nq * L::kTileBytes));
+      for (int t = 0; t < nq; ++t)
+        for (int s = 0; s < L::kSub; ++s)
+          tma_load_3d(smem + L::kQOff + t * L::kTileBytes + s * L::kSubBytes, &tm_q, q_full, s * 64,
+                      q0_row + t * 128, bh, pol_q);
+      for (int j = 0; j < nmax; ++j) {
+        const int st = j % L::kStages;
+        if (!mbar_wait(&kv_empty[st], ((j / L::kStages) & 1) ^ 1, wd)) break;
+        mbar_arrive_expect_tx(&kv_full[st], uint32_t(2 * L::kTileBytes));
+        uint8_t* sk = smem + L::kKVOff + st * 2 * L::kTileBytes;
+        uint8_t* sv = sk + L::kTileBytes;
+        for (int s = 0; s < L::kSub; ++s) {
+          tma_load_3d(sk + s * L::kSubBytes, &tm_k, &kv_full[st], s * 64, j * 128, bh, pol_kv);
+          tma_load_3d(sv + s * L::kSubBytes, &tm_v, &kv_full[st], s * 64, j * 128, bh, pol_kv);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = make_idesc_bf16(128, 128, 0, 0);   // Q K^T: both K-major
+      constexpr uint32_t kIdPV = make_idesc_bf16(128, D, 0, 1);    // P_bar V: V is MN-major
+      const uint32_t sq = smem_u32(smem + L::kQOff);
+      const uint32_t skv = smem_u32(smem + L::kKVOff);
+      auto issue_s = [&](int t, int st) {
+        const uint32_t qa = sq + t * L::kTileBytes;
+        const uint32_t ka = skv + st * 2 * L::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * L::kSubBytes + (k & 3) * 32;
+          umma_ss(tmem + t * 128, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
+                  kIdS, k > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int st, int j) {
+        const uint32_t va = skv + st * 2 * L::kTileBytes + L::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_ts(tmem + 256 + t * D, tmem + t * 128 + k * 8, make_sdesc_sw128(va + k * 2048, L::kSubBytes, 1024),
+                  kIdPV, (j > 0 || k > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(q_full, 0, wd) && mbar_wait(&kv_full[0], 0, wd);
+      if (ok) {
+        tc_fence_after();
+        if (n0 > 0) { issue_s(0, 0); umma_commit(&s_full[0]); }
+        if (n1 > 0) { issue_s(1, 0); umma_commit(&s_full[1]); }
+      }
+      for (int j = 0; ok && j < nmax; ++j) {
+        const int st = j % L::kStages;
+        const int jn = j + 1;
+        const int stn = jn % L::kStages;
+        if (j < n0) {
+          if (!(ok = mbar_wait(&p_full[0], j & 1, wd))) break;
+          tc_fence_after();
+          issue_pv(0, st, j);
+          umma_commit(&o_done[0]);
+        }
+        if (jn < nmax) {
+          if (!(ok = mbar_wait(&kv_full[stn], (jn / L::kStages) & 1, wd))) break;
+          tc_fence_after();
+        }
+        if (jn < n0) { issue_s(0, stn); umma_commit(&s_full[0]); }
+        if (j < n1) {
+          if (!(ok = mbar_wait(&p_full[1], j & 1, wd))) break;
+          tc_fence_after();
+          issue_pv(1, st, j);
+          umma_commit(&o_done[1]);
+        }
+        umma_commit(&kv_empty[st]);
+        if (jn < n1) { issue_s(1, stn); umma_commit(&s_full[1]); }
+      }
+      // Every MMA must be finished before TMEM is released.
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, wd);
+    }
+    __syncwarp();
+  } else {
+    // --------------------------------------------------- softmax warpgroups
+    const int t = warp >> 2;
+    const int n_t = t ? n1 : n0;
+    const int row = (t ? q1_row : q0_row) + (warp & 3) * 32 + lane;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + uint32_t(t * 128);
+    const uint32_t t_o = tmem + lane_base + uint32_t(256 + t * D);
+    const int limit = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
+
+    float m = kNegInf;    // running max of the raw scores S
+    int cnt = 0;          // how many seen scores equal m
+    float ms = kNegInf;   // shift in use, base-2 exponent units (m*scale_log2 [+ delta])
+    float l = 0.f;        // running sum of the unrounded P
+    bool ok = true;
+
+    for (int j = 0; j < n_t; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wd));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, r[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_wait(r[c]);
+      float s[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(r[i >> 5][i & 31]);
+
+      const int key0 = j * 128;
+      if (key0 + 127 > limit) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) s[i] = (key0 + i > limit) ? kNegInf : s[i];
+      }
+      // tile maximum and how often it occurs (exact FP32 equality)
+      float mt0 = s[0], mt1 = s[1], mt2 = s[2], mt3 = s[3];
+#pragma unroll
+      for (int i = 4; i < 128; i += 4) {
+        mt0 = fmaxf(mt0, s[i]);
+        mt1 = fmaxf(mt1, s[i + 1]);
+        mt2 = fmaxf(mt2, s[i + 2]);
+        mt3 = fmaxf(mt3, s[i + 3]);
+      }
+      const float mt = fmaxf(fmaxf(mt0, mt1), fmaxf(mt2, mt3));
+      int ct = 0;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) ct += (s[i] == mt) ? 1 : 0;
+      const float m_new = fmaxf(m, mt);
+      int c_new = (m == m_new ? cnt : 0) + (mt == m_new ? ct : 0);
+      if (m_new == kNegInf) c_new = 0;
+      const bool repeated = p.fix && c_new >= 2;
+      const float ms_new = (m_new == kNegInf) ? 0.f : fmaf(m_new, p.scale_log2, repeated ? p.delta_log2 : 0.f);
+      const float alpha = ex2(ms - ms_new);
+
+      // P = 2^(S*scale_log2 - ms_new); l sums P, the MMA gets bf16(P)
+      float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2(fmaf(s[c * 32 + 2 * i], p.scale_log2, -ms_new));
+          const float p1 = ex2(fmaf(s[c * 32 + 2 * i + 1], p.scale_log2, -ms_new));
+          rs0 += p0;
+          rs1 += p1;
+          pk[i] = pack_bf16(p0, p1);
+        }
+        tmem_st16(t_s + c * 16, pk);
+      }
+      l = l * alpha + (rs0 + rs1);
+      tmem_st_wait();
+
+      if (j > 0) {
+        // O_t must hold the finished P_bar V of tile j-1 before it is rescaled
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (j - 1) & 1, wd));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, ms_new != ms)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c * 32, o);
+            tmem_ld_wait(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_o + c * 32, o);
+          }
+          tmem_st_wait();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+      m = m_new;
+      cnt = c_new;
+      ms = ms_new;
+    }
+
+    if (ok && n_t > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (n_t - 1) & 1, wd));
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        __nv_bfloat16* orow = p.o + (size_t(bh) * p.N + row) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c * 32, o);
+          tmem_ld_wait(o);
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+          if (row < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
+        }
+        if (row < p.N) {
+          p.lse[size_t(bh) * p.N + row] = (ms + lg2(l)) * kLn2;
+          if (p.ties) p.ties[size_t(bh) * p.N + row] = cnt;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,171 @@
+"""Thin ctypes binding of libfa_b200.so (include/fa_b200.h).
+
+Argument marshalling only: every step of attention runs in the library's CUDA
+kernels.  Tensors are torch tensors on a CUDA device (torch provides memory
+and streams); there is no CPU path.  Importing this module loads the library
+and raises if it has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "FAError", "LIB_PATH", "lib", "fa_fwd", "fa_fwd_ties", "fa_bwd", "fa_bwd_workspace_size",
+    "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish",
+    "fa_status_string", "fa_check_device_error", "EXPORTED", "attention_fwd", "attention_bwd",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
+
+FA_OK = 0
+EXPORTED = ("fa_fwd", "fa_fwd_ties", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
+            "fa_bwd_finish", "fa_status_string", "fa_check_device_error")
+
+
+class FAError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        self.status = status
+        super().__init__(f"{call} failed: {status} ({fa_status_string(status)})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m flashattention_bf16_fwd_b200.build` "
+            "(there is no CPU fallback)")
+    so = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    so.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    so.fa_fwd.restype = i
+    so.fa_fwd_ties.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    so.fa_fwd_ties.restype = i
+    so.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    so.fa_bwd_workspace_size.restype = sz
+    so.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, vp]
+    so.fa_bwd.restype = i
+    so.fa_bwd_preprocess.argtypes = [vp, vp, vp, sz, i, i, i, i, vp]
+    so.fa_bwd_preprocess.restype = i
+    so.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, vp]
+    so.fa_bwd_main.restype = i
+    so.fa_bwd_finish.argtypes = [vp, vp, sz, i, i, i, i, f, vp]
+    so.fa_bwd_finish.restype = i
+    so.fa_status_string.argtypes = [i]
+    so.fa_status_string.restype = ctypes.c_char_p
+    so.fa_check_device_error.argtypes = [vp]
+    so.fa_check_device_error.restype = i
+    return so
+
+
+lib = _load()
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device (the library has no CPU path)")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _shape(q):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    return tuple(int(x) for x in q.shape)
+
+
+def fa_status_string(status: int) -> str:
+    return lib.fa_status_string(int(status)).decode()
+
+
+def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, fix_mode: int, stream=None) -> int:
+    B, H, N, d = _shape(q)
+    return lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, int(causal), float(scale),
+                      int(fix_mode), _stream(stream))
+
+
+def fa_fwd_ties(q, k, v, o, lse, ties, causal: bool, scale: float, fix_mode: int, stream=None) -> int:
+    B, H, N, d = _shape(q)
+    return lib.fa_fwd_ties(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(ties), B, H, N, d, int(causal),
+                           float(scale), int(fix_mode), _stream(stream))
+
+
+def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(lib.fa_bwd_workspace_size(B, H, N, d))
+
+
+def fa_bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool, scale: float, stream=None) -> int:
+    B, H, N, d = _shape(q)
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                      _ptr(workspace), nbytes, B, H, N, d, int(causal), float(scale), _stream(stream))
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size() if t is not None else 0
+
+
+def fa_bwd_preprocess(o, do, workspace, stream=None) -> int:
+    B, H, N, d = _shape(o)
+    return lib.fa_bwd_preprocess(_ptr(o), _ptr(do), _ptr(workspace), _nbytes(workspace), B, H, N, d,
+                                 _stream(stream))
+
+
+def fa_bwd_main(q, k, v, lse, do, dk, dv, workspace, causal: bool, scale: float, stream=None) -> int:
+    B, H, N, d = _shape(q)
+    return lib.fa_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(lse), _ptr(do), _ptr(dk), _ptr(dv), _ptr(workspace),
+                           _nbytes(workspace), B, H, N, d, int(causal), float(scale), _stream(stream))
+
+
+def fa_bwd_finish(dq, workspace, scale: float, stream=None) -> int:
+    B, H, N, d = _shape(dq)
+    return lib.fa_bwd_finish(_ptr(dq), _ptr(workspace), _nbytes(workspace), B, H, N, d, float(scale),
+                             _stream(stream))
+
+
+def fa_check_device_error(stream=None) -> int:
+    return lib.fa_check_device_error(_stream(stream))
+
+
+def _check(call: str, status: int):
+    if status != FA_OK:
+        raise FAError(call, status)
+
+
+def attention_fwd(q, k, v, causal: bool = True, scale: float | None = None, fix_mode: int = 1,
+                  stream=None, ties: bool = False):
+    """Allocate O and LSE (and optionally the per-row tie counts) and run fa_fwd."""
+    B, H, N, d = _shape(q)
+    scale = d ** -0.5 if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if ties:
+        t = torch.empty((B, H, N), dtype=torch.int32, device=q.device)
+        _check("fa_fwd_ties", fa_fwd_ties(q, k, v, o, lse, t, causal, scale, fix_mode, stream))
+        return o, lse, t
+    _check("fa_fwd", fa_fwd(q, k, v, o, lse, causal, scale, fix_mode, stream))
+    return o, lse
+
+
+def attention_bwd(q, k, v, o, lse, do, causal: bool = True, scale: float | None = None, stream=None,
+                  workspace=None):
+    """Allocate dQ, dK, dV (and the workspace unless given) and run fa_bwd."""
+    B, H, N, d = _shape(q)
+    scale = d ** -0.5 if scale is None else scale
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=q.device)
+    _check("fa_bwd", fa_bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal, scale, stream))
+    return dq, dk, dv

@@ -1,0 +1,153 @@
+/*
+ * fa_b200.h - C ABI of the B200 (sm_100a) BF16 FlashAttention library.
+ *
+ * What the calls compute (the statement of attention on the pages):
+ *   S = scale * Q K^T, P = softmax(S) row by row, O = P V
+ *   ("Is Flash Attention Stable?", chibakuma.com: the standard/baseline
+ *   attention that FlashAttention reorders with tiling and kernel fusion),
+ * evaluated the FlashAttention way: K/V tiles streamed through shared memory,
+ * an online safe softmax with a running row maximum m and row sum l, the
+ * unnormalised output P_bar V accumulated in FP32 and divided by l at the end,
+ * and the log-sum-exp kept for a backward pass that recomputes P
+ * (yicaiai article, abstract and sections 1.1, 3.4, 4.3).
+ *
+ * The repeated-max fix ("Why Low-Precision Transformer Training Fails: An
+ * Analysis on Flash Attention", admirer.cn summary, "mechanism 2"): per row,
+ * detect whether the maximum of S occurs more than once; if it does, raise
+ * the safe-softmax shift m so that every exponent, the ones at the maximum
+ * included, is strictly below 1.  This library raises m by
+ * delta = -log2(1 - 2^-8) in the base-2 exponent domain, which maps each
+ * maximum to exactly 1 - 2^-8 = 0.99609375, the largest bf16 value below 1.
+ * P_bar is rounded to bf16 (round to nearest even) before the P_bar V
+ * product; l sums the unrounded FP32 P.
+ *
+ * Conventions shared by every call
+ *   - Tensors Q, K, V, O, dO, dQ, dK, dV are bf16, contiguous [B, H, N, d]
+ *     (row-major, d fastest).  LSE is float32 [B, H, N] in natural-log units.
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller; the
+ *     library never allocates, frees or keeps a pointer after a call returns.
+ *     Base addresses must be 16-byte aligned (TMA requirement).
+ *   - d is 64 or 128.  N >= 1, any value (ragged tails are masked).  B, H >= 1.
+ *     B*H*N*d must be below 2^31.  scale must be finite and > 0.
+ *   - causal: 0 = every key visible; 1 = key j visible to query i iff j <= i.
+ *   - stream is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous on it; the return value reports argument and launch
+ *     errors only.  Kernel-side watchdog timeouts are reported by
+ *     fa_check_device_error().
+ *   - On any error nothing is launched and outputs are left untouched.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_NULL = -1,      /* a required pointer is NULL                       */
+  FA_ERR_SHAPE = -2,     /* B, H or N < 1, or B*H*N*d too large               */
+  FA_ERR_HEADDIM = -3,   /* d not in {64, 128}                                */
+  FA_ERR_ALIGN = -4,     /* a tensor base is not 16-byte aligned              */
+  FA_ERR_FIXMODE = -5,   /* fix_mode not in {0, 1}                            */
+  FA_ERR_WORKSPACE = -6, /* workspace NULL, misaligned or too small           */
+  FA_ERR_LAUNCH = -7,    /* the CUDA runtime refused a launch                 */
+  FA_ERR_TIMEOUT = -8,   /* a kernel's bounded wait expired (device flag)     */
+  FA_ERR_ARG = -9,       /* causal not in {0,1}, or scale not finite and > 0  */
+  FA_ERR_DEVICE = -10    /* no sm_100 device, or the driver entry point for
+                            tensor maps is unavailable                        */
+} fa_status;
+
+/*
+ * fa_fwd - attention forward pass with the optional repeated-max fix.
+ *   q, k, v  in : bf16 [B,H,N,d], device.
+ *   o        out: bf16 [B,H,N,d], device.  O = (P_bar V) / l, rounded to bf16.
+ *   lse      out: float32 [B,H,N], device.  LSE_i = log sum_j exp(S_ij).
+ *   fix_mode    : 0 = plain safe softmax (shift = row max);
+ *                 1 = repeated-max fix as described above.
+ * Returns FA_OK or a negative fa_status.
+ */
+FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int H, int N, int d, int causal, float scale, int fix_mode,
+           void* stream);
+
+/*
+ * fa_fwd_ties - fa_fwd plus a per-row record of the repeated-max detector:
+ *   ties out: int32 [B,H,N], device.  The number of visible keys whose FP32
+ *             score equals the row maximum of S (>= 2 means the fix fired
+ *             when fix_mode == 1).  Same kernel as fa_fwd; the extra store
+ *             is one int per row.
+ */
+FA_API int fa_fwd_ties(const void* q, const void* k, const void* v, void* o, float* lse,
+                int32_t* ties, int B, int H, int N, int d, int causal,
+                float scale, int fix_mode, void* stream);
+
+/*
+ * fa_bwd_workspace_size - bytes of device scratch fa_bwd needs:
+ *   an FP32 dQ accumulator [B,H,N,d] and FP32 D_i = sum_k dO_ik O_ik [B,H,N].
+ * Returns 0 for invalid shapes.
+ */
+FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * fa_bwd - attention backward pass that recomputes P from the LSE.
+ *   q, k, v, o, dout in : bf16 [B,H,N,d], device (o and lse from fa_fwd).
+ *   lse              in : float32 [B,H,N], device.
+ *   dq, dk, dv       out: bf16 [B,H,N,d], device.
+ *   workspace        tmp: device, >= fa_bwd_workspace_size() bytes, 16-byte
+ *                         aligned; contents on entry are ignored.
+ * Gradients of sum(dO * O): dV = P^T dO, dS = P * (dO V^T - D),
+ * dQ = scale dS K, dK = scale dS^T Q.  No fix_mode argument: LSE does not
+ * depend on the shift, so the recomputed P is the same either way.
+ */
+FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o,
+           const float* lse, const void* dout, void* dq, void* dk, void* dv,
+           void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+           int causal, float scale, void* stream);
+
+/*
+ * The three launches fa_bwd makes, callable one by one (same arguments and
+ * checks as fa_bwd; all three must see the same workspace, in this order):
+ *   fa_bwd_preprocess  D_i = sum_k dO_ik O_ik into the workspace, and a zeroed
+ *                      FP32 dQ accumulator (reads O and dO once).
+ *   fa_bwd_main        recompute P per (key tile, query tile), write dK and dV,
+ *                      and add the unscaled dQ contributions into the
+ *                      accumulator.
+ *   fa_bwd_finish      dQ = scale * accumulator, rounded to bf16.
+ */
+FA_API int fa_bwd_preprocess(const void* o, const void* dout, void* workspace,
+                             size_t workspace_bytes, int B, int H, int N, int d,
+                             void* stream);
+FA_API int fa_bwd_main(const void* q, const void* k, const void* v,
+                       const float* lse, const void* dout, void* dk, void* dv,
+                       void* workspace, size_t workspace_bytes, int B, int H,
+                       int N, int d, int causal, float scale, void* stream);
+FA_API int fa_bwd_finish(void* dq, const void* workspace, size_t workspace_bytes,
+                         int B, int H, int N, int d, float scale, void* stream);
+
+/* fa_status_string - static, NUL-terminated description of a status code. */
+FA_API const char* fa_status_string(int status);
+
+/*
+ * fa_check_device_error - synchronises `stream`, then reads and clears the
+ * library's device error flag on the current device.  Returns FA_OK,
+ * FA_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last check,
+ * FA_ERR_DEVICE if a kernel found its shared memory misaligned and did no
+ * work, or FA_ERR_LAUNCH if the stream reports a CUDA error.
+ */
+FA_API int fa_check_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

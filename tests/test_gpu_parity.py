@@ -1,0 +1,223 @@
+"""GPU parity: the CUDA path (through the C ABI) against the FP64 oracle.
+
+Tolerances (stated for N(0,1) inputs):
+  O     max |O_gpu - O_ref|                               <= 2e-2
+  LSE   max |LSE_gpu - LSE_ref| / max(|LSE_ref|, 1)        <= 1e-3
+  dQ, dK, dV  ||X_gpu - X_ref||_F / ||X_ref||_F           <= 5e-2
+Small shapes are compared element by element over every head; the full-size
+workloads run exactly as bench.py launches them and are compared on sampled
+(batch, head) pairs, each against a whole-head oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from flashattention_bf16_fwd_b200.stats import bias_stats, lse_rel_err, normwise_rel_err
+from flashattention_bf16_fwd_b200.workloads import WORKLOADS, Workload, make_inputs
+from oracle import attention_bwd, attention_fwd, attention_fwd_bf16p, tie_counts
+
+pytestmark = pytest.mark.gpu
+
+O_ATOL = 2e-2
+LSE_RTOL = 1e-3
+GRAD_RTOL = 5e-2
+
+
+@pytest.fixture(scope="module")
+def fa():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from flashattention_bf16_fwd_b200 import fa as binding
+    return binding
+
+
+def run_gpu(fa, x, fix_mode=1, bwd=True, ties=False, heads=None):
+    dev = torch.device("cuda")
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    res = fa.attention_fwd(q, k, v, causal=x["causal"], scale=x["scale"], fix_mode=fix_mode, ties=ties)
+    out = {"o": res[0], "lse": res[1]}
+    if ties:
+        out["ties"] = res[2]
+    if bwd:
+        dq, dk, dv = fa.attention_bwd(q, k, v, res[0], res[1], x["do"].to(dev), causal=x["causal"], scale=x["scale"])
+        out.update(dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    assert fa.fa_check_device_error() == 0
+    sel = (slice(None), slice(None)) if heads is None else heads
+    return {n: t[sel].float().cpu().numpy() if t.dtype != torch.int32 else t[sel].cpu().numpy()
+            for n, t in out.items()}
+
+
+def sub(x, b, h):
+    return {n: (t[b:b + 1, h:h + 1] if torch.is_tensor(t) else t) for n, t in x.items()}
+
+
+def check_fwd(g, x):
+    o_ref, lse_ref = attention_fwd(x["q"], x["k"], x["v"], x["causal"], x["scale"])
+    err_o = np.abs(g["o"] - o_ref).max()
+    err_l = lse_rel_err(g["lse"], lse_ref)
+    assert np.isfinite(g["o"]).all() and np.isfinite(g["lse"]).all()
+    assert err_o <= O_ATOL, err_o
+    assert err_l <= LSE_RTOL, err_l
+    return err_o, err_l
+
+
+def check_bwd(g, x):
+    ref = attention_bwd(x["q"], x["k"], x["v"], x["do"], x["causal"], x["scale"])
+    errs = {}
+    for name, r in zip(("dq", "dk", "dv"), ref):
+        assert np.isfinite(g[name]).all(), name
+        errs[name] = normwise_rel_err(g[name], r)
+        assert errs[name] <= GRAD_RTOL, (name, errs[name])
+    return errs
+
+
+SHAPES = [  # B, H, N, d, causal
+    (1, 1, 1, 64, 1),
+    (1, 2, 127, 64, 1),
+    (2, 1, 129, 64, 0),
+    (1, 2, 256, 64, 1),
+    (1, 1, 200, 128, 1),
+    (1, 2, 384, 128, 0),
+    (2, 2, 256, 128, 1),
+    (1, 2, 1000, 64, 1),
+    (1, 1, 1000, 128, 0),
+    (1, 1, 641, 64, 0),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", SHAPES, ids=[f"B{b}H{h}N{n}d{d}{'c' if c else 'f'}" for b, h, n, d, c in SHAPES])
+@pytest.mark.parametrize("fix_mode", [0, 1])
+def test_fwd_bwd_shapes(fa, B, H, N, d, causal, fix_mode):
+    w = Workload("shape", B, H, N, d, causal=bool(causal))
+    x = make_inputs(w, seed=N + d + causal)
+    g = run_gpu(fa, x, fix_mode=fix_mode)
+    check_fwd(g, x)
+    check_bwd(g, x)
+
+
+@pytest.mark.parametrize("fix_mode", [0, 1])
+def test_tiny_workload(fa, fix_mode):
+    x = make_inputs(WORKLOADS["tiny"], seed=0)
+    g = run_gpu(fa, x, fix_mode=fix_mode, ties=True)
+    check_fwd(g, x)
+    check_bwd(g, x)
+    # the emulated oracle (bf16 P_bar with one shift per row) is closer still
+    oe, _ = attention_fwd_bf16p(x["q"], x["k"], x["v"], True, x["scale"], fix_mode)
+    assert np.abs(g["o"] - oe).max() <= O_ATOL
+
+
+def test_tie_counts_match_oracle(fa):
+    for w in (WORKLOADS["tiny"], WORKLOADS["long"].with_shape(B=1, H=4, N=1024),
+              WORKLOADS["gpt2m"].with_shape(B=1, H=2, N=512)):
+        x = make_inputs(w, seed=3, with_grad=False)
+        g = run_gpu(fa, x, fix_mode=1, bwd=False, ties=True)
+        ref = tie_counts(x["q"], x["k"], w.causal)
+        rep = ref >= 2
+        assert rep.sum() > 0
+        # repeated maxima built from copied keys are exact in FP32 as in FP64
+        assert np.array_equal(g["ties"][rep], ref[rep])
+        # elsewhere a coincidence of two distinct FP32 scores is allowed, rarely
+        assert np.mean(g["ties"][~rep] == 1) > 0.999
+
+
+def test_fix_changes_only_repeated_rows(fa):
+    x = make_inputs(WORKLOADS["long"].with_shape(B=1, H=4, N=1024), seed=5, with_grad=False)
+    g0 = run_gpu(fa, x, fix_mode=0, bwd=False, ties=True)
+    g1 = run_gpu(fa, x, fix_mode=1, bwd=False, ties=True)
+    assert np.array_equal(g0["ties"], g1["ties"])
+    rep = g1["ties"] >= 2
+    same = np.all(g0["o"] == g1["o"], axis=-1)
+    # rows that never saw a repeated maximum run the identical arithmetic
+    assert np.mean(same[~rep]) > 0.97
+    assert not np.all(same[rep])
+
+
+def test_deterministic_forward(fa):
+    x = make_inputs(WORKLOADS["tiny"].with_shape(B=2, H=3, N=700), seed=9)
+    a = run_gpu(fa, x, bwd=True)
+    b = run_gpu(fa, x, bwd=True)
+    for n in ("o", "lse", "dk", "dv"):
+        assert np.array_equal(a[n], b[n]), n
+    # dQ is summed with atomics in an arbitrary order: equal up to rounding
+    assert normwise_rel_err(a["dq"], b["dq"]) < 1e-5
+
+
+def test_outputs_stay_in_bounds(fa):
+    """Guard regions around every output keep their NaN canary."""
+    B, H, N, d = 1, 2, 333, 128
+    x = make_inputs(Workload("g", B, H, N, d), seed=11)
+    dev = torch.device("cuda")
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    G = 4096
+
+    def guarded(shape, dtype):
+        n = int(np.prod(shape))
+        buf = torch.full((n + 2 * G,), float("nan"), dtype=dtype, device=dev)
+        return buf, buf[G:G + n].view(shape)
+
+    bo, o = guarded((B, H, N, d), torch.bfloat16)
+    bl, lse = guarded((B, H, N), torch.float32)
+    assert fa.fa_fwd(q, k, v, o, lse, True, x["scale"], 1) == 0
+    bufs = [guarded((B, H, N, d), torch.bfloat16) for _ in range(3)]
+    wsz = fa.fa_bwd_workspace_size(B, H, N, d)
+    bw = torch.full((wsz + 2 * G,), 0x7F, dtype=torch.uint8, device=dev)
+    ws = bw[G:G + wsz]
+    assert fa.fa_bwd(q, k, v, o, lse, do, bufs[0][1], bufs[1][1], bufs[2][1], ws, True, x["scale"]) == 0
+    torch.cuda.synchronize()
+    assert fa.fa_check_device_error() == 0
+    for buf, view in [(bo, o), (bl, lse)] + bufs:
+        assert torch.isnan(buf[:G]).all() and torch.isnan(buf[-G:]).all()
+        assert torch.isfinite(view).all()
+    assert (bw[:G] == 0x7F).all() and (bw[-G:] == 0x7F).all()
+
+
+FULL = ["gpt2s", "gpt2m", "long", "llama7b"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_heads(fa, name):
+    w = WORKLOADS[name]
+    x = make_inputs(w, seed=0)
+    rng = np.random.default_rng(123)
+    picks = [(int(rng.integers(w.B)), int(rng.integers(w.H))) for _ in range(2)]
+    dev = torch.device("cuda")
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, lse = fa.attention_fwd(q, k, v, causal=w.causal, scale=w.scale, fix_mode=1)
+    dq, dk, dv = fa.attention_bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    assert fa.fa_check_device_error() == 0
+    for b, h in picks:
+        g = {n: t[b:b + 1, h:h + 1].float().cpu().numpy()
+             for n, t in dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv).items()}
+        xs = sub(x, b, h)
+        check_fwd(g, xs)
+        check_bwd(g, xs)
+    # every output finite, everywhere
+    for t in (o, lse, dq, dk, dv):
+        assert torch.isfinite(t).all()
+
+
+def test_no_sign_coherent_bias_with_fix(fa):
+    """Repeated-max rows: the fix leaves no sign-coherent error in O.
+
+    e = O_gpu - O_exact on rows whose maximum of S repeats.  Per row r the mean
+    error and the magnitude-aligned mean sign(O_exact) * e are the independent
+    samples.  With fix_mode = 1 both means must be within 3 standard errors of
+    zero and the aligned mean below 2^-12 mean|O_exact|.  fix_mode = 0 is
+    measured alongside and printed.
+    """
+    w = WORKLOADS["long"].with_shape(B=2, H=8, N=2048)
+    x = make_inputs(w, seed=1, with_grad=False)
+    o_ref, _ = attention_fwd(x["q"], x["k"], x["v"], True, w.scale)
+    ref_ties = tie_counts(x["q"], x["k"], True)
+    rep = ref_ties >= 2
+    assert rep.sum() > 1000
+    out = {}
+    for fix in (0, 1):
+        g = run_gpu(fa, x, fix_mode=fix, bwd=False)
+        out[fix] = bias_stats(g["o"], o_ref, rep)
+        out[f"control{fix}"] = bias_stats(g["o"], o_ref, ~rep)
+    print("bias on repeated-max rows:", out)
+    s = out[1]
+    assert abs(s["z_mean"]) < 3 and abs(s["z_aligned"]) < 3
+    assert abs(s["aligned_mean"]) <= 2.0 ** -12 * s["mean_abs_ref"]
