@@ -211,6 +211,7 @@ __global__ void __launch_bounds__(320, 1)
     int cnt = 0;          // how many seen scores equal m
     float ms = kNegInf;   // shift in use, base-2 exponent units (m*scale_log2 [+ delta])
     float l = 0.f;        // running sum of the unrounded P
+    bool ever_repeated = false;   // the running max occurred >= 2 times at some tile
     bool ok = true;
 
     for (int j = 0; j < n_t; ++j) {
@@ -247,6 +248,7 @@ __global__ void __launch_bounds__(320, 1)
       const float m_new = fmaxf(m, mt);
       int c_new = (m == m_new ? cnt : 0) + (mt == m_new ? ct : 0);
       if (m_new == kNegInf) c_new = 0;
+      ever_repeated |= (c_new >= 2);
       const bool repeated = p.fix && c_new >= 2;
       const float ms_new = (m_new == kNegInf) ? 0.f : fmaf(m_new, p.scale_log2, repeated ? p.delta_log2 : 0.f);
       const float alpha = ex2(ms - ms_new);
@@ -317,7 +319,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (row < p.N) {
           p.lse[size_t(bh) * p.N + row] = (ms + lg2(l)) * kLn2;
-          if (p.ties) p.ties[size_t(bh) * p.N + row] = cnt;
+          if (p.ties) p.ties[size_t(bh) * p.N + row] = cnt | (ever_repeated ? (1 << 30) : 0);
         }
       }
     }

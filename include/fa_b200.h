@@ -82,10 +82,13 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* l
 
 /*
  * fa_fwd_ties - fa_fwd plus a per-row record of the repeated-max detector:
- *   ties out: int32 [B,H,N], device.  The number of visible keys whose FP32
- *             score equals the row maximum of S (>= 2 means the fix fired
- *             when fix_mode == 1).  Same kernel as fa_fwd; the extra store
- *             is one int per row.
+ *   ties out: int32 [B,H,N], device.  Bits 0-29: the number of visible keys
+ *             whose FP32 score equals the row maximum of S (>= 2 means the
+ *             fix applies to the final shift when fix_mode == 1).  Bit 30:
+ *             set if the running maximum was repeated at any key tile, i.e.
+ *             the detector fired at some point of the row (with fix_mode 1
+ *             the shift was raised then).  Same kernel as fa_fwd; the extra
+ *             store is one int per row.
  */
 FA_API int fa_fwd_ties(const void* q, const void* k, const void* v, void* o, float* lse,
                 int32_t* ties, int B, int H, int N, int d, int causal,

@@ -23,3 +23,9 @@ def test_error_measures():
     assert abs(max_rel_err(x, ref) - 0.05) < 1e-12
     assert abs(normwise_rel_err(x, ref) - np.sqrt(0.05) / np.sqrt(1 + 4 + 0.25 + 16)) < 1e-12
     assert abs(lse_rel_err([0.0005, 10.01], [0.0, 10.0]) - 1e-3) < 1e-12
+
+
+def test_normwise_floor_for_vanishing_gradients():
+    ref = np.zeros((4, 64))
+    assert normwise_rel_err(ref + 1e-8, ref) < 1e-4
+    assert normwise_rel_err(ref + 1e-3, ref) >= 0.99
