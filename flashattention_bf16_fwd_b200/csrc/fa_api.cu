@@ -63,6 +63,17 @@ DeviceState* device_state() {
                                FwdLayout<64>::kAlloc) == cudaSuccess;
     ok &= cudaFuncSetAttribute(fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                FwdLayout<128>::kAlloc) == cudaSuccess;
+    // The forward kernel moves registers between warpgroups with setmaxnreg;
+    // the split assumes exactly kLaunchRegs registers per thread at launch.
+    cudaFuncAttributes fattr{};
+    ok &= cudaFuncGetAttributes(&fattr, fa_fwd_kernel<64>) == cudaSuccess &&
+          fattr.numRegs == FwdLayout<64>::kLaunchRegs;
+    ok &= cudaFuncGetAttributes(&fattr, fa_fwd_kernel<128>) == cudaSuccess &&
+          fattr.numRegs == FwdLayout<128>::kLaunchRegs;
+    ok &= cudaFuncGetAttributes(&fattr, fa_bwd_kernel<64>) == cudaSuccess &&
+          fattr.numRegs == BwdLayout<64>::kLaunchRegs;
+    ok &= cudaFuncGetAttributes(&fattr, fa_bwd_kernel<128>) == cudaSuccess &&
+          fattr.numRegs == BwdLayout<128>::kLaunchRegs;
     ok &= cudaFuncSetAttribute(fa_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                BwdLayout<64>::kAlloc) == cudaSuccess;
     ok &= cudaFuncSetAttribute(fa_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -94,6 +105,20 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The FP32 dQ accumulator [BH, N, D] as 3-D (d, n, bh) with 32 x 32 boxes and
+// the 128-byte swizzle, for TMA reduce-add.
+bool make_map_dq(CUtensorMap* map, const void* base, int BH, int N, int D) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(N), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(D) * 4, cuuint64_t(N) * D * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -196,9 +221,9 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, c
   if (!st) return FA_ERR_DEVICE;
   const int BH = B * H;
   const size_t rows = size_t(BH) * N;
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   if (!make_map(&mq, q, BH, N, d) || !make_map(&mk, k, BH, N, d) || !make_map(&mv, v, BH, N, d) ||
-      !make_map(&mdo, dout, BH, N, d))
+      !make_map(&mdo, dout, BH, N, d) || !make_map_dq(&mdq, workspace, BH, N, d))
     return FA_ERR_DEVICE;
   BwdParams prm{};
   prm.lse = lse;
@@ -216,9 +241,9 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, c
   const dim3 grid(unsigned(prm.n_kv) * unsigned(BH));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
-    fa_bwd_kernel<64><<<grid, BwdLayout<64>::kThreads, BwdLayout<64>::kAlloc, s>>>(mq, mk, mv, mdo, prm);
+    fa_bwd_kernel<64><<<grid, BwdLayout<64>::kThreads, BwdLayout<64>::kAlloc, s>>>(mq, mk, mv, mdo, mdq, prm);
   else
-    fa_bwd_kernel<128><<<grid, BwdLayout<128>::kThreads, BwdLayout<128>::kAlloc, s>>>(mq, mk, mv, mdo, prm);
+    fa_bwd_kernel<128><<<grid, BwdLayout<128>::kThreads, BwdLayout<128>::kAlloc, s>>>(mq, mk, mv, mdo, mdq, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 

@@ -10,17 +10,10 @@
 //   fa_bwd_kernel      one CTA per (batch*head, 128-key tile); loops over the
 //                      query tiles that see those keys; five tcgen05 MMAs per
 //                      step; dK, dV stay in TMEM; dQ is added into the FP32
-//                      accumulator with vector atomics
+//                      accumulator with TMA reduce-add from shared memory
 //   fa_bwd_dq_kernel   dQ = scale * accumulator -> bf16 (HBM-bound)
 //
-// fa_bwd_kernel warp roles (320 threads):
-//   warps 0-3  key-row math: thread r owns key r (TMEM lane r); P^T, dS^T
-//   warps 4-7  dQ drain (thread r owns query r of the tile) and the dK/dV
-//              epilogue
-//   warp  8    producer: K, V once; Q_i, dO_i (TMA) plus LSE_i, D_i per step
-//   warp  9    TMEM allocator + tcgen05.mma issuer
-// TMEM: S^T [0,128) (P_bar^T aliases [0,64)), dP^T [128,256) (dS^T aliases
-// [128,192)), dV, dK, then dQ (d=64) or dQ aliasing dP^T (d=128).
+// fa_bwd_kernel roles and TMEM use are described above the kernel.
 #pragma once
 
 #include "sm100.cuh"
@@ -97,25 +90,54 @@ struct BwdLayout {
   static constexpr int kTileBytes = kSub * kSubBytes;
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kTileBytes;
+  static constexpr int kDOStages = (D == 64) ? 2 : 1;      // d=128: one dO buffer, refilled after dV
   static constexpr int kQOff = 2 * kTileBytes;             // 2 stages
-  static constexpr int kDOOff = kQOff + 2 * kTileBytes;    // 2 stages
-  static constexpr int kDSOff = kDOOff + 2 * kTileBytes;   // dS, [128 keys][128 queries] bf16, MN-major
-  static constexpr int kStatOff = kDSOff + 2 * kSubBytes;  // 2 stages x (LSE*log2e, D) x 128 floats
-  static constexpr int kBarOff = kStatOff + 2 * 2 * 128 * 4;
+  static constexpr int kDOOff = kQOff + 2 * kTileBytes;
+  static constexpr int kDSOff = kDOOff + kDOStages * kTileBytes;   // dS, [128 keys][128 queries] bf16, MN-major
+  static constexpr int kStatOff = kDSOff + 2 * kSubBytes;  // 2 stages x (-LSE*log2e, D) x 128 floats
+  // dQ staging for the TMA reduce-add: per drain warp two 32 x 32 FP32 boxes
+  static constexpr int kStageBox = 32 * 32 * 4;
+  static constexpr int kDQStageOff = kStatOff + 2 * 2 * 128 * 4;
+  static constexpr int kBarOff = kDQStageOff + 4 * 2 * kStageBox;
   static constexpr int kBytes = kBarOff + 256;
   static constexpr int kAlloc = kBytes;                    // base is 1 KB aligned by declaration
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kThreads = 320;
-  static constexpr bool kDqAliasDp = (D == 128);
+  static constexpr int kThreads = 512;
+  static constexpr int kLaunchRegs = 128;                  // per thread, fixed by __launch_bounds__(512, 1)
+  static constexpr uint32_t kComputeRegs = 168;
+  static constexpr uint32_t kDrainRegs = 104;
+  static constexpr uint32_t kOtherRegs = 72;
+  static_assert(128 * (2 * kComputeRegs + kDrainRegs + kOtherRegs) <= kThreads * kLaunchRegs,
+                "register split exceeds the pool");
+  // TMEM columns.  d = 64: P_bar^T has its own 64 columns, so S of the next
+  // query tile can be computed while this tile's dS is formed.  d = 128: no
+  // room; P_bar^T overwrites half of each S half and dQ reuses dP^T.
+  static constexpr bool kWide = (D == 128);
   static constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDV = 256, kTmDK = 256 + D;
-  static constexpr uint32_t kTmDQ = kDqAliasDp ? 128 : 256 + 2 * D;
+  static constexpr uint32_t kTmDQ = kWide ? 128 : 384;
+  static constexpr uint32_t kTmPT = kWide ? 0 : 448;
+  // column of P_bar^T / dS^T for MMA K-step k (16 queries = 8 columns): the
+  // query half h = k / 4 was written by the warps that own that half
+  __host__ __device__ static constexpr uint32_t pt_col(int k) { return kWide ? kTmS + 64 * (k >> 2) + 8 * (k & 3) : kTmPT + 8 * k; }
+  __host__ __device__ static constexpr uint32_t dst_col(int k) { return kTmDP + 64 * (k >> 2) + 8 * (k & 3); }
 };
 
+// Roles (16 warps):
+//   warps 0-7   key-row math; warp w owns keys 32*(w%4).. (TMEM lane quarter
+//               w%4) and queries 64*(w/4).. of each tile: P^T, dS^T
+//   warps 8-11  dQ drain (thread r owns query r; TMA reduce-add of 32 x 32
+//               FP32 boxes staged in shared memory) and the dK/dV epilogue
+//   warp  12    producer: K, V once; Q_i, dO_i (TMA) plus LSE_i, D_i per step
+//   warp  13    TMEM allocator + tcgen05.mma issuer
+//   warps 14-15 idle (complete the fourth warpgroup)
+// MMA order per query tile i (the tensor core runs the next tile's S while
+// the CUDA cores form dS_i, and dK_i, dQ_i, dP_{i+1} while they form P_{i+1}):
+//   dV_i += P_bar_i^T dO_i | S_{i+1} | dK_i += dS_i^T Q_i | dQ_i = dS_i K | dP_{i+1}
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using L = BwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
@@ -129,9 +151,12 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* dq_full = bars + 9;
   uint64_t* dq_free = bars + 10;
   uint64_t* dkv_done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* pt_free = bars + 12;
+  uint64_t* do_full = bars + 13;   // [2]
+  uint64_t* do_empty = bars + 15;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* stats = reinterpret_cast<float*>(smem + L::kStatOff);   // [stage][lse2 | dsum][128]
+  float* stats = reinterpret_cast<float*>(smem + L::kStatOff);   // [stage][-lse2 | dsum][128]
 
   // The 128-byte swizzle needs 1 KB aligned tiles; the layout has no room to
   // realign, so a misaligned dynamic shared-memory base is reported, not used.
@@ -155,24 +180,30 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&q_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(p_full, 256);
     mbar_init(dp_full, 1);
-    mbar_init(ds_full, 128);
+    mbar_init(ds_full, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 128);
     mbar_init(dkv_done, 1);
+    mbar_init(pt_free, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&do_full[s], 1);
+      mbar_init(&do_empty[s], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
   }
   tc_fence_before();
   __syncthreads();
@@ -180,144 +211,190 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.dev_error};
 
-  if (warp == 8) {
-    // ------------------------------------------------------------- producer
-    const uint64_t pol_kv = l2_policy_evict_first();
-    const uint64_t pol_q = l2_policy_evict_last();
-    if (lane == 0) {
-      mbar_arrive_expect_tx(kv_full, uint32_t(2 * L::kTileBytes));
-      for (int s = 0; s < L::kSub; ++s) {
-        tma_load_3d(smem + L::kKOff + s * L::kSubBytes, &tm_k, kv_full, s * 64, key0, bh, pol_kv);
-        tma_load_3d(smem + L::kVOff + s * L::kSubBytes, &tm_v, kv_full, s * 64, key0, bh, pol_kv);
-      }
-    }
-    const float kLog2e = 1.4426950408889634f;
-    for (int it = 0; it < n_it; ++it) {
-      const int st = it & 1;
-      const int q0 = (i_start + it) * 128;
-      if (!__all_sync(0xffffffffu, mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1, wd))) break;
-      float* lse2 = stats + st * 256;
-      float* dd = lse2 + 128;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = lane * 4 + u;
-        const int row = q0 + r;
-        const bool in = row < p.N;
-        lse2[r] = in ? p.lse[size_t(bh) * p.N + row] * kLog2e : __int_as_float(0x7f800000);
-        dd[r] = in ? p.dsum[size_t(bh) * p.N + row] : 0.f;
-      }
-      __syncwarp();
+  if (warp >= 12) {
+    // Producer and MMA warps need few registers; give them back first.
+    regs_decrease<L::kOtherRegs>();
+    if (warp == 12) {
+      // ----------------------------------------------------------- producer
+      const uint64_t pol_kv = l2_policy_evict_first();
+      const uint64_t pol_q = l2_policy_evict_last();
       if (lane == 0) {
-        mbar_arrive_expect_tx(&q_full[st], uint32_t(2 * L::kTileBytes));
+        mbar_arrive_expect_tx(kv_full, uint32_t(2 * L::kTileBytes));
         for (int s = 0; s < L::kSub; ++s) {
-          tma_load_3d(smem + L::kQOff + st * L::kTileBytes + s * L::kSubBytes, &tm_q, &q_full[st], s * 64, q0, bh,
-                      pol_q);
-          tma_load_3d(smem + L::kDOOff + st * L::kTileBytes + s * L::kSubBytes, &tm_do, &q_full[st], s * 64, q0,
-                      bh, pol_q);
+          tma_load_3d(smem + L::kKOff + s * L::kSubBytes, &tm_k, kv_full, s * 64, key0, bh, pol_kv);
+          tma_load_3d(smem + L::kVOff + s * L::kSubBytes, &tm_v, kv_full, s * 64, key0, bh, pol_kv);
         }
+      }
+      const float kLog2e = 1.4426950408889634f;
+      for (int it = 0; it < n_it; ++it) {
+        const int st = it & 1;
+        const int q0 = (i_start + it) * 128;
+        if (!__all_sync(0xffffffffu, mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1, wd))) break;
+        float* nlse = stats + st * 256;
+        float* dd = nlse + 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = lane * 4 + u;
+          const int row = q0 + r;
+          const bool in = row < p.N;
+          // rows past N: P = 2^(-inf) = 0 and D = 0, so they add nothing
+          nlse[r] = in ? -p.lse[size_t(bh) * p.N + row] * kLog2e : -__int_as_float(0x7f800000);
+          dd[r] = in ? p.dsum[size_t(bh) * p.N + row] : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&q_full[st], uint32_t(L::kTileBytes));
+          for (int s = 0; s < L::kSub; ++s)
+            tma_load_3d(smem + L::kQOff + st * L::kTileBytes + s * L::kSubBytes, &tm_q, &q_full[st], s * 64, q0,
+                        bh, pol_q);
+        }
+        // dO_i: with a single buffer it is refilled once dV_{i-1} has read it
+        const int sd = it % L::kDOStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(&do_empty[sd], ((it / L::kDOStages) & 1) ^ 1, wd))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&do_full[sd], uint32_t(L::kTileBytes));
+          for (int s = 0; s < L::kSub; ++s)
+            tma_load_3d(smem + L::kDOOff + sd * L::kTileBytes + s * L::kSubBytes, &tm_do, &do_full[sd], s * 64, q0,
+                        bh, pol_q);
+        }
+        __syncwarp();
+      }
+    } else if (warp == 13) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t kIdS = make_idesc_bf16(128, 128, 0, 0);   // K Q^T, V dO^T: K-major operands
+        constexpr uint32_t kIdAcc = make_idesc_bf16(128, D, 0, 1);   // TMEM A x MN-major B (dV, dK)
+        constexpr uint32_t kIdDQ = make_idesc_bf16(128, D, 1, 1);    // dS (MN-major) x K (MN-major)
+        const uint32_t sk = smem_u32(smem + L::kKOff);
+        const uint32_t sv = smem_u32(smem + L::kVOff);
+        const uint32_t sds = smem_u32(smem + L::kDSOff);
+        auto kmajor_mma = [&](uint32_t d_tm, uint32_t a, uint32_t b) {
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k >> 2) * L::kSubBytes + (k & 3) * 32;
+            umma_ss(d_tm, make_sdesc_sw128(a + off, 16, 1024), make_sdesc_sw128(b + off, 16, 1024), kIdS, k > 0);
+          }
+        };
+        auto q_of = [&](int it) { return smem_u32(smem + L::kQOff + (it & 1) * L::kTileBytes); };
+        auto do_of = [&](int it) { return smem_u32(smem + L::kDOOff + (it % L::kDOStages) * L::kTileBytes); };
+        auto wait_do = [&](int it) {
+          return mbar_wait(&do_full[it % L::kDOStages], (it / L::kDOStages) & 1, wd);
+        };
+        bool ok = mbar_wait(kv_full, 0, wd) && mbar_wait(&q_full[0], 0, wd) && wait_do(0);
+        if (ok) {
+          tc_fence_after();
+          kmajor_mma(tmem + L::kTmS, sk, q_of(0));     // S^T_0 = K Q_0^T
+          umma_commit(s_full);
+          kmajor_mma(tmem + L::kTmDP, sv, do_of(0));   // dP^T_0 = V dO_0^T
+          umma_commit(dp_full);
+        }
+        for (int it = 0; ok && it < n_it; ++it) {
+          const uint32_t sq = q_of(it);
+          const uint32_t sdo = do_of(it);
+          if (!(ok = mbar_wait(p_full, it & 1, wd))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)                   // dV += P_bar^T dO_i
+            umma_ts(tmem + L::kTmDV, tmem + L::pt_col(k), make_sdesc_sw128(sdo + k * 2048, L::kSubBytes, 1024),
+                    kIdAcc, (it > 0 || k > 0) ? 1u : 0u);
+          umma_commit(pt_free);
+          umma_commit(&do_empty[it % L::kDOStages]);    // dP_i and dV_i were the readers of dO_i
+          if (it + 1 < n_it) {                          // S^T_{i+1}
+            if (!(ok = mbar_wait(&q_full[(it + 1) & 1], ((it + 1) >> 1) & 1, wd))) break;
+            tc_fence_after();
+            kmajor_mma(tmem + L::kTmS, sk, q_of(it + 1));
+            umma_commit(s_full);
+          }
+          if (!(ok = mbar_wait(ds_full, it & 1, wd))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)                   // dK += dS^T Q_i
+            umma_ts(tmem + L::kTmDK, tmem + L::dst_col(k), make_sdesc_sw128(sq + k * 2048, L::kSubBytes, 1024),
+                    kIdAcc, (it > 0 || k > 0) ? 1u : 0u);
+          if (!L::kWide && it > 0) {                    // the drain has read dQ_{i-1}
+            if (!(ok = mbar_wait(dq_free, (it - 1) & 1, wd))) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k)                   // dQ_i = dS K
+            umma_ss(tmem + L::kTmDQ, make_sdesc_sw128(sds + k * 2048, L::kSubBytes, 1024),
+                    make_sdesc_sw128(sk + k * 2048, L::kSubBytes, 1024), kIdDQ, k > 0 ? 1u : 0u);
+          umma_commit(dq_full);
+          umma_commit(&q_empty[it & 1]);
+          if (it + 1 < n_it) {                          // dP^T_{i+1}
+            if (L::kWide) {                             // dQ_i shares the dP^T columns
+              if (!(ok = mbar_wait(dq_free, it & 1, wd))) break;
+              tc_fence_after();
+            }
+            if (!(ok = wait_do(it + 1))) break;
+            tc_fence_after();
+            kmajor_mma(tmem + L::kTmDP, sv, do_of(it + 1));
+            umma_commit(dp_full);
+          }
+        }
+        umma_commit(dkv_done);
+        mbar_wait(dkv_done, 0, wd);
       }
       __syncwarp();
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdS = make_idesc_bf16(128, 128, 0, 0);   // K Q^T, V dO^T: K-major operands
-      constexpr uint32_t kIdAcc = make_idesc_bf16(128, D, 0, 1);   // TMEM A x MN-major B (dV, dK)
-      constexpr uint32_t kIdDQ = make_idesc_bf16(128, D, 1, 1);    // dS (MN-major) x K (MN-major)
-      const uint32_t sk = smem_u32(smem + L::kKOff);
-      const uint32_t sv = smem_u32(smem + L::kVOff);
-      const uint32_t sds = smem_u32(smem + L::kDSOff);
-      auto kmajor_mma = [&](uint32_t d_tm, uint32_t a, uint32_t b) {
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * L::kSubBytes + (k & 3) * 32;
-          umma_ss(d_tm, make_sdesc_sw128(a + off, 16, 1024), make_sdesc_sw128(b + off, 16, 1024), kIdS, k > 0);
-        }
-      };
-      bool ok = mbar_wait(kv_full, 0, wd);
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int st = it & 1;
-        const uint32_t sq = smem_u32(smem + L::kQOff + st * L::kTileBytes);
-        const uint32_t sdo = smem_u32(smem + L::kDOOff + st * L::kTileBytes);
-        if (!(ok = mbar_wait(&q_full[st], (it >> 1) & 1, wd))) break;
-        tc_fence_after();
-        kmajor_mma(tmem + L::kTmS, sk, sq);            // S^T = K Q_i^T
-        umma_commit(s_full);
-        if (L::kDqAliasDp && it > 0) {                  // dQ_{i-1} shares columns with dP^T
-          if (!(ok = mbar_wait(dq_free, (it - 1) & 1, wd))) break;
-          tc_fence_after();
-        }
-        kmajor_mma(tmem + L::kTmDP, sv, sdo);          // dP^T = V dO_i^T
-        umma_commit(dp_full);
-        if (!(ok = mbar_wait(p_full, it & 1, wd))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 8; ++k)                     // dV += P_bar^T dO_i
-          umma_ts(tmem + L::kTmDV, tmem + L::kTmS + k * 8, make_sdesc_sw128(sdo + k * 2048, L::kSubBytes, 1024),
-                  kIdAcc, (it > 0 || k > 0) ? 1u : 0u);
-        if (!(ok = mbar_wait(ds_full, it & 1, wd))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 8; ++k)                     // dK += dS^T Q_i
-          umma_ts(tmem + L::kTmDK, tmem + L::kTmDP + k * 8, make_sdesc_sw128(sq + k * 2048, L::kSubBytes, 1024),
-                  kIdAcc, (it > 0 || k > 0) ? 1u : 0u);
-        if (!L::kDqAliasDp && it > 0) {
-          if (!(ok = mbar_wait(dq_free, (it - 1) & 1, wd))) break;
-          tc_fence_after();
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k)                     // dQ_i = dS K
-          umma_ss(tmem + L::kTmDQ, make_sdesc_sw128(sds + k * 2048, L::kSubBytes, 1024),
-                  make_sdesc_sw128(sk + k * 2048, L::kSubBytes, 1024), kIdDQ, k > 0 ? 1u : 0u);
-        umma_commit(dq_full);
-        umma_commit(&q_empty[st]);
-      }
-      umma_commit(dkv_done);
-      mbar_wait(dkv_done, 0, wd);
-    }
-    __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
+    regs_increase<L::kComputeRegs>();
     // ------------------------------------------------------- key-row math
-    const int kr = warp * 32 + lane;                 // key within the tile
+    const int quarter = warp & 3;
+    const int half = warp >> 2;                      // queries 64*half .. +63
+    const int kr = quarter * 32 + lane;              // key within the tile
     const int key = key0 + kr;
     const bool key_in = key < p.N;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    const uint32_t t_s = tmem + lane_base + L::kTmS;
-    const uint32_t t_dp = tmem + lane_base + L::kTmDP;
-    uint8_t* ds_row = smem + L::kDSOff + kr * 128;
+    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + L::kTmS + 64 * half;
+    const uint32_t t_dp = tmem + lane_base + L::kTmDP + 64 * half;
+    const uint32_t t_pt = tmem + lane_base + (L::kWide ? L::kTmS + 64 * half : L::kTmPT + 32 * half);
+    uint8_t* ds_row = smem + L::kDSOff + half * L::kSubBytes + kr * 128;
+    const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     for (int it = 0; it < n_it; ++it) {
       const int st = it & 1;
       const int qt = i_start + it;
-      const float* lse2 = stats + st * 256;
-      const float* dd = lse2 + 128;
+      const float* nlse = stats + st * 256 + 64 * half;
+      const float* dd = stats + st * 256 + 128 + 64 * half;
       // q_full publishes this stage's LSE/D (written by the producer's lanes)
       if (!__all_sync(0xffffffffu, mbar_wait(&q_full[st], (it >> 1) & 1, wd))) break;
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, it & 1, wd))) break;
       tc_fence_after();
-      // P^T row: P[q] = 2^(S*scale_log2 - LSE2[q]); masked entries are 0
-      uint32_t pk[64];
-      const bool diag = p.causal && qt == kv_tile;
+      // P^T: P[q] = 2^(S*scale_log2 - LSE2[q]); masked entries are 0
+      uint32_t pk[32];
+      {
+        uint32_t r[2][32];
+        tmem_ld32(t_s, r[0]);
+        tmem_ld32(t_s + 32, r[1]);
+        tmem_ld_wait(r[0]);
+        tmem_ld_wait(r[1]);
+        const bool diag = p.causal && qt == kv_tile;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_s + c * 32, r);
-        tmem_ld_wait(r);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int q = c * 32 + i;
-          float p0 = ex2(fmaf(__uint_as_float(r[i]), p.scale_log2, -lse2[q]));
-          float p1 = ex2(fmaf(__uint_as_float(r[i + 1]), p.scale_log2, -lse2[q + 1]));
-          if (!key_in || (diag && q < kr)) p0 = 0.f;
-          if (!key_in || (diag && q + 1 < kr)) p1 = 0.f;
-          pk[(c * 32 + i) >> 1] = pack_bf16(p0, p1);
+        for (int i = 0; i < 32; ++i) {
+          const int q = 2 * i;                         // query within this half
+          const uint64_t nl = *reinterpret_cast<const uint64_t*>(nlse + q);
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
+                                   __uint_as_float(r[i >> 4][(2 * i + 1) & 31])), c2, nl), x0, x1);
+          float p0 = ex2(x0), p1 = ex2(x1);
+          const int qg = 64 * half + q;                // query within the tile
+          if (!key_in || (diag && qg < kr)) p0 = 0.f;
+          if (!key_in || (diag && qg + 1 < kr)) p1 = 0.f;
+          pk[i] = pack_bf16(p0, p1);
         }
       }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      if (!L::kWide && it > 0) {                       // dV_{i-1} has read P_bar^T_{i-1}
+        if (!__all_sync(0xffffffffu, mbar_wait(pt_free, (it - 1) & 1, wd))) break;
+        tc_fence_after();
+      }
+      {
         uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = pk[c * 16 + i];
-        tmem_st16(t_s + c * 16, w);
+        for (int i = 0; i < 16; ++i) w[i] = pk[i];
+        tmem_st16(t_pt, w);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = pk[16 + i];
+        tmem_st16(t_pt + 16, w);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -325,38 +402,42 @@ __global__ void __launch_bounds__(320, 1)
 
       if (!__all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, wd))) break;
       tc_fence_after();
-      // dS^T row = P_bar * (dP - D[q])
-      uint32_t dk_w[64];
+      // dS^T = P_bar * (dP - D[q])
+      uint32_t dsw[32];
+      {
+        uint32_t r[2][32];
+        tmem_ld32(t_dp, r[0]);
+        tmem_ld32(t_dp + 32, r[1]);
+        tmem_ld_wait(r[0]);
+        tmem_ld_wait(r[1]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_dp + c * 32, r);
-        tmem_ld_wait(r);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int q = c * 32 + i;
-          const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[q >> 1]));
-          const float d0 = pp.x * (__uint_as_float(r[i]) - dd[q]);
-          const float d1 = pp.y * (__uint_as_float(r[i + 1]) - dd[q + 1]);
-          dk_w[q >> 1] = pack_bf16(d0, d1);
+        for (int i = 0; i < 32; ++i) {
+          const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[i]));
+          const uint64_t dq2 = *reinterpret_cast<const uint64_t*>(dd + 2 * i);
+          const uint64_t dp2 = f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
+                                       __uint_as_float(r[i >> 4][(2 * i + 1) & 31]));
+          float y0, y1;
+          f2_unpack(f2_mul(f2_fma(dq2, f2_pack(-1.f, -1.f), dp2), f2_pack(pp.x, pp.y)), y0, y1);
+          dsw[i] = pack_bf16(y0, y1);
         }
       }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      {
         uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = dk_w[c * 16 + i];
-        tmem_st16(t_dp + c * 16, w);
+        for (int i = 0; i < 16; ++i) w[i] = dsw[i];
+        tmem_st16(t_dp, w);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = dsw[16 + i];
+        tmem_st16(t_dp + 16, w);
       }
       // dS into shared memory for dQ = dS K: MN-major, 128-byte swizzle
       if (it > 0) {
         if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (it - 1) & 1, wd))) break;
       }
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int blk = ch >> 3, c16 = ch & 7;
-        uint4* dst = reinterpret_cast<uint4*>(ds_row + blk * L::kSubBytes + ((c16 ^ (kr & 7)) << 4));
-        *dst = make_uint4(dk_w[ch * 4], dk_w[ch * 4 + 1], dk_w[ch * 4 + 2], dk_w[ch * 4 + 3]);
+      for (int c16 = 0; c16 < 8; ++c16) {
+        uint4* dst = reinterpret_cast<uint4*>(ds_row + ((c16 ^ (kr & 7)) << 4));
+        *dst = make_uint4(dsw[c16 * 4], dsw[c16 * 4 + 1], dsw[c16 * 4 + 2], dsw[c16 * 4 + 3]);
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tmem_st_wait();
@@ -364,33 +445,46 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(ds_full);
     }
   } else {
+    regs_decrease<L::kDrainRegs>();
     // ------------------------------------------- dQ drain and dK/dV epilogue
     const int wq = warp & 3;
     const int rr = wq * 32 + lane;                   // query row (dQ) / key row (dK, dV)
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
     const uint32_t t_dq = tmem + lane_base + L::kTmDQ;
+    uint8_t* stage = smem + L::kDQStageOff + wq * 2 * L::kStageBox;
+    uint32_t box_seq = 0;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      const int row = (i_start + it) * 128 + rr;
       ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, wd));
       if (!ok) break;
       tc_fence_after();
-      float4* dst = reinterpret_cast<float4*>(p.dq_acc + (size_t(bh) * p.N + row) * D);
+      // TMEM -> swizzled 32 x 32 FP32 box in shared memory -> TMA reduce-add
+      // into the FP32 accumulator (rows past N are dropped by the TMA unit)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(t_dq + c * 32, r);
         tmem_ld_wait(r);
-        if (row < p.N) {
+        uint8_t* box = stage + (box_seq & 1) * L::kStageBox;
+        if (lane == 0) bulk_wait_read<1>();              // the reduce issued from this box is done reading
+        __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            atomicAdd(dst + c * 8 + i, make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                                   __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
+        for (int c16 = 0; c16 < 8; ++c16)
+          *reinterpret_cast<uint4*>(box + lane * 128 + ((c16 ^ (lane & 7)) << 4)) =
+              make_uint4(r[4 * c16], r[4 * c16 + 1], r[4 * c16 + 2], r[4 * c16 + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tm_dq, box, c * 32, (i_start + it) * 128 + wq * 32, bh);
+          bulk_commit();
         }
+        ++box_seq;
       }
       tc_fence_before();
       mbar_arrive(dq_free);
     }
+    if (lane == 0) bulk_wait<0>();                      // every reduce-add has landed
+    __syncwarp();
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dkv_done, 0, wd));
     if (ok) {
       tc_fence_after();
@@ -421,7 +515,7 @@ __global__ void __launch_bounds__(320, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }

@@ -16,6 +16,10 @@
 //   warps 4-7  softmax of query tile 1
 //   warp  8    TMA producer: Q tiles once, then a ring of K/V stages
 //   warp  9    TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 10-11 idle (they complete the third warpgroup)
+// Registers: launched at 168 per thread (384 threads); the third warpgroup
+// gives back down to 56 and the two softmax warpgroups take 224 each:
+// 128 * (224 + 224 + 56) = 384 * 168.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 after.
 // P_bar (bf16, two per 32-bit column) overwrites the first 64 columns of S_t
 // and is the A operand of O_t += P_bar V (V is the MN-major B operand).
@@ -48,11 +52,15 @@ struct FwdLayout {
   static constexpr int kBytes = kBarOff + 256;
   static constexpr int kAlloc = kBytes + 1024;        // room to align the base to 1 KB
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 384;
+  static constexpr int kLaunchRegs = 168;       // per thread, fixed by __launch_bounds__(384, 1)
+  static constexpr uint32_t kSoftmaxRegs = 224;
+  static constexpr uint32_t kOtherRegs = 56;
+  static_assert(128 * (2 * kSoftmaxRegs + kOtherRegs) <= kThreads * kLaunchRegs, "register split exceeds the pool");
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using L = FwdLayout<D>;
@@ -115,89 +123,94 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.dev_error};
 
-  if (warp == 8) {
-    // ------------------------------------------------------------- producer
-    if (lane == 0) {
-      const uint64_t pol_q = l2_policy_evict_first();
-      const uint64_t pol_kv = l2_policy_evict_last();
-      const int nq = (n1 > 0) ? 2 : 1;
-      mbar_arrive_expect_tx(q_full, uint32_t(nq * L::kTileBytes));
-      for (int t = 0; t < nq; ++t)
-        for (int s = 0; s < L::kSub; ++s)
-          tma_load_3d(smem + L::kQOff + t * L::kTileBytes + s * L::kSubBytes, &tm_q, q_full, s * 64,
-                      q0_row + t * 128, bh, pol_q);
-      for (int j = 0; j < nmax; ++j) {
-        const int st = j % L::kStages;
-        if (!mbar_wait(&kv_empty[st], ((j / L::kStages) & 1) ^ 1, wd)) break;
-        mbar_arrive_expect_tx(&kv_full[st], uint32_t(2 * L::kTileBytes));
-        uint8_t* sk = smem + L::kKVOff + st * 2 * L::kTileBytes;
-        uint8_t* sv = sk + L::kTileBytes;
-        for (int s = 0; s < L::kSub; ++s) {
-          tma_load_3d(sk + s * L::kSubBytes, &tm_k, &kv_full[st], s * 64, j * 128, bh, pol_kv);
-          tma_load_3d(sv + s * L::kSubBytes, &tm_v, &kv_full[st], s * 64, j * 128, bh, pol_kv);
+  if (warp >= 8) {
+    // Producer and MMA warps need few registers; give them back first.
+    regs_decrease<L::kOtherRegs>();
+    if (warp == 8) {
+      // ------------------------------------------------------------- producer
+      if (lane == 0) {
+        const uint64_t pol_q = l2_policy_evict_first();
+        const uint64_t pol_kv = l2_policy_evict_last();
+        const int nq = (n1 > 0) ? 2 : 1;
+        mbar_arrive_expect_tx(q_full, uint32_t(nq * L::kTileBytes));
+        for (int t = 0; t < nq; ++t)
+          for (int s = 0; s < L::kSub; ++s)
+            tma_load_3d(smem + L::kQOff + t * L::kTileBytes + s * L::kSubBytes, &tm_q, q_full, s * 64,
+                        q0_row + t * 128, bh, pol_q);
+        for (int j = 0; j < nmax; ++j) {
+          const int st = j % L::kStages;
+          if (!mbar_wait(&kv_empty[st], ((j / L::kStages) & 1) ^ 1, wd)) break;
+          mbar_arrive_expect_tx(&kv_full[st], uint32_t(2 * L::kTileBytes));
+          uint8_t* sk = smem + L::kKVOff + st * 2 * L::kTileBytes;
+          uint8_t* sv = sk + L::kTileBytes;
+          for (int s = 0; s < L::kSub; ++s) {
+            tma_load_3d(sk + s * L::kSubBytes, &tm_k, &kv_full[st], s * 64, j * 128, bh, pol_kv);
+            tma_load_3d(sv + s * L::kSubBytes, &tm_v, &kv_full[st], s * 64, j * 128, bh, pol_kv);
+          }
         }
       }
+    } else if (warp == 9) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t kIdS = make_idesc_bf16(128, 128, 0, 0);   // Q K^T: both K-major
+        constexpr uint32_t kIdPV = make_idesc_bf16(128, D, 0, 1);    // P_bar V: V is MN-major
+        const uint32_t sq = smem_u32(smem + L::kQOff);
+        const uint32_t skv = smem_u32(smem + L::kKVOff);
+        auto issue_s = [&](int t, int st) {
+          const uint32_t qa = sq + t * L::kTileBytes;
+          const uint32_t ka = skv + st * 2 * L::kTileBytes;
+  #pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k >> 2) * L::kSubBytes + (k & 3) * 32;
+            umma_ss(tmem + t * 128, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
+                    kIdS, k > 0);
+          }
+        };
+        auto issue_pv = [&](int t, int st, int j) {
+          const uint32_t va = skv + st * 2 * L::kTileBytes + L::kTileBytes;
+  #pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_ts(tmem + 256 + t * D, tmem + t * 128 + k * 8, make_sdesc_sw128(va + k * 2048, L::kSubBytes, 1024),
+                    kIdPV, (j > 0 || k > 0) ? 1u : 0u);
+        };
+        bool ok = mbar_wait(q_full, 0, wd) && mbar_wait(&kv_full[0], 0, wd);
+        if (ok) {
+          tc_fence_after();
+          if (n0 > 0) { issue_s(0, 0); umma_commit(&s_full[0]); }
+          if (n1 > 0) { issue_s(1, 0); umma_commit(&s_full[1]); }
+        }
+        for (int j = 0; ok && j < nmax; ++j) {
+          const int st = j % L::kStages;
+          const int jn = j + 1;
+          const int stn = jn % L::kStages;
+          if (j < n0) {
+            if (!(ok = mbar_wait(&p_full[0], j & 1, wd))) break;
+            tc_fence_after();
+            issue_pv(0, st, j);
+            umma_commit(&o_done[0]);
+          }
+          if (jn < nmax) {
+            if (!(ok = mbar_wait(&kv_full[stn], (jn / L::kStages) & 1, wd))) break;
+            tc_fence_after();
+          }
+          if (jn < n0) { issue_s(0, stn); umma_commit(&s_full[0]); }
+          if (j < n1) {
+            if (!(ok = mbar_wait(&p_full[1], j & 1, wd))) break;
+            tc_fence_after();
+            issue_pv(1, st, j);
+            umma_commit(&o_done[1]);
+          }
+          umma_commit(&kv_empty[st]);
+          if (jn < n1) { issue_s(1, stn); umma_commit(&s_full[1]); }
+        }
+        // Every MMA must be finished before TMEM is released.
+        umma_commit(mma_done);
+        mbar_wait(mma_done, 0, wd);
+      }
+      __syncwarp();
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdS = make_idesc_bf16(128, 128, 0, 0);   // Q K^T: both K-major
-      constexpr uint32_t kIdPV = make_idesc_bf16(128, D, 0, 1);    // P_bar V: V is MN-major
-      const uint32_t sq = smem_u32(smem + L::kQOff);
-      const uint32_t skv = smem_u32(smem + L::kKVOff);
-      auto issue_s = [&](int t, int st) {
-        const uint32_t qa = sq + t * L::kTileBytes;
-        const uint32_t ka = skv + st * 2 * L::kTileBytes;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * L::kSubBytes + (k & 3) * 32;
-          umma_ss(tmem + t * 128, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
-                  kIdS, k > 0);
-        }
-      };
-      auto issue_pv = [&](int t, int st, int j) {
-        const uint32_t va = skv + st * 2 * L::kTileBytes + L::kTileBytes;
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          umma_ts(tmem + 256 + t * D, tmem + t * 128 + k * 8, make_sdesc_sw128(va + k * 2048, L::kSubBytes, 1024),
-                  kIdPV, (j > 0 || k > 0) ? 1u : 0u);
-      };
-      bool ok = mbar_wait(q_full, 0, wd) && mbar_wait(&kv_full[0], 0, wd);
-      if (ok) {
-        tc_fence_after();
-        if (n0 > 0) { issue_s(0, 0); umma_commit(&s_full[0]); }
-        if (n1 > 0) { issue_s(1, 0); umma_commit(&s_full[1]); }
-      }
-      for (int j = 0; ok && j < nmax; ++j) {
-        const int st = j % L::kStages;
-        const int jn = j + 1;
-        const int stn = jn % L::kStages;
-        if (j < n0) {
-          if (!(ok = mbar_wait(&p_full[0], j & 1, wd))) break;
-          tc_fence_after();
-          issue_pv(0, st, j);
-          umma_commit(&o_done[0]);
-        }
-        if (jn < nmax) {
-          if (!(ok = mbar_wait(&kv_full[stn], (jn / L::kStages) & 1, wd))) break;
-          tc_fence_after();
-        }
-        if (jn < n0) { issue_s(0, stn); umma_commit(&s_full[0]); }
-        if (j < n1) {
-          if (!(ok = mbar_wait(&p_full[1], j & 1, wd))) break;
-          tc_fence_after();
-          issue_pv(1, st, j);
-          umma_commit(&o_done[1]);
-        }
-        umma_commit(&kv_empty[st]);
-        if (jn < n1) { issue_s(1, stn); umma_commit(&s_full[1]); }
-      }
-      // Every MMA must be finished before TMEM is released.
-      umma_commit(mma_done);
-      mbar_wait(mma_done, 0, wd);
-    }
-    __syncwarp();
   } else {
+    regs_increase<L::kSoftmaxRegs>();
     // --------------------------------------------------- softmax warpgroups
     const int t = warp >> 2;
     const int n_t = t ? n1 : n0;
@@ -206,11 +219,17 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t t_s = tmem + lane_base + uint32_t(t * 128);
     const uint32_t t_o = tmem + lane_base + uint32_t(256 + t * D);
     const int limit = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
+    const float sl2 = p.scale_log2;
+    // 2^-delta: on a repeated-max row P is computed with the plain shift and
+    // then multiplied by this, which is the same as raising m by delta; each
+    // maximum lands exactly on 1 - 2^-8.
+    const float kFixFactor = 0.99609375f;
 
     float m = kNegInf;    // running max of the raw scores S
     int cnt = 0;          // how many seen scores equal m
-    float ms = kNegInf;   // shift in use, base-2 exponent units (m*scale_log2 [+ delta])
-    float l = 0.f;        // running sum of the unrounded P
+    float ms = kNegInf;   // m * scale_log2: the shift without the fix
+    bool raised = false;  // the shift in use is ms + delta (fix active on this row)
+    float l = 0.f;        // running sum of the unrounded P, relative to the shift in use
     bool ever_repeated = false;   // the running max occurred >= 2 times at some tile
     bool ok = true;
 
@@ -228,47 +247,82 @@ __global__ void __launch_bounds__(320, 1)
       for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(r[i >> 5][i & 31]);
 
       const int key0 = j * 128;
-      if (key0 + 127 > limit) {
+      const bool masked = key0 + 127 > limit;
+      if (masked) {
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = (key0 + i > limit) ? kNegInf : s[i];
       }
-      // tile maximum and how often it occurs (exact FP32 equality)
-      float mt0 = s[0], mt1 = s[1], mt2 = s[2], mt3 = s[3];
+      // tile maximum: eight 16-wide 3-input max chains, then a short tree
+      float mx[8];
 #pragma unroll
-      for (int i = 4; i < 128; i += 4) {
-        mt0 = fmaxf(mt0, s[i]);
-        mt1 = fmaxf(mt1, s[i + 1]);
-        mt2 = fmaxf(mt2, s[i + 2]);
-        mt3 = fmaxf(mt3, s[i + 3]);
+      for (int g = 0; g < 8; ++g) {
+        float a = fmax3(s[16 * g], s[16 * g + 1], s[16 * g + 2]);
+#pragma unroll
+        for (int i = 3; i < 15; i += 2) a = fmax3(a, s[16 * g + i], s[16 * g + i + 1]);
+        mx[g] = fmaxf(a, s[16 * g + 15]);
       }
-      const float mt = fmaxf(fmaxf(mt0, mt1), fmaxf(mt2, mt3));
-      int ct = 0;
-#pragma unroll
-      for (int i = 0; i < 128; ++i) ct += (s[i] == mt) ? 1 : 0;
+      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
       const float m_new = fmaxf(m, mt);
+      const float ms_new = (m_new == kNegInf) ? 0.f : m_new * sl2;
+
+      // P = 2^(S*scale_log2 - ms_new) in pairs; row sum and the count of
+      // entries equal to the tile max ride along as independent adds
+      const uint64_t c2 = f2_pack(sl2, sl2);
+      const uint64_t b2 = f2_pack(-ms_new, -ms_new);
+      uint64_t sum2[4] = {0, 0, 0, 0};
+      uint64_t eq2[2] = {0, 0};
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float x0 = fmaf(s[2 * i], sl2, -ms_new);
+        const float x1 = fmaf(s[2 * i + 1], sl2, -ms_new);
+        const float e0 = (s[2 * i] == mt) ? 1.f : 0.f;
+        const float e1 = (s[2 * i + 1] == mt) ? 1.f : 0.f;
+        eq2[i & 1] = f2_add(eq2[i & 1], f2_pack(e0, e1));
+        s[2 * i] = ex2(x0);
+        s[2 * i + 1] = ex2(x1);
+        sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(s[2 * i], s[2 * i + 1]));
+      }
+      float ea, eb, ec, ed;
+      f2_unpack(f2_add(eq2[0], eq2[1]), ea, eb);
+      const int ct = (mt == kNegInf) ? 0 : int(ea + eb);
       int c_new = (m == m_new ? cnt : 0) + (mt == m_new ? ct : 0);
       if (m_new == kNegInf) c_new = 0;
       ever_repeated |= (c_new >= 2);
-      const bool repeated = p.fix && c_new >= 2;
-      const float ms_new = (m_new == kNegInf) ? 0.f : fmaf(m_new, p.scale_log2, repeated ? p.delta_log2 : 0.f);
-      const float alpha = ex2(ms - ms_new);
-
-      // P = 2^(S*scale_log2 - ms_new); l sums P, the MMA gets bf16(P)
-      float rs0 = 0.f, rs1 = 0.f;
+      const bool raise = p.fix && c_new >= 2;
+      f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), ea, eb);
+      float rs = ea + eb;
+      if (__any_sync(0xffffffffu, raise)) {
+        // Rare path: some row of this warp has a repeated maximum.  S is still
+        // intact in TMEM; recompute P for the whole warp (unchanged rows get
+        // the identical arithmetic) and scale the repeated rows by 2^-delta.
+        uint32_t q[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, q[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_wait(q[c]);
+        float rs_raised = 0.f;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const float sv = (masked && key0 + i > limit) ? kNegInf : __uint_as_float(q[i >> 5][i & 31]);
+          const float pv = ex2(fmaf(sv, sl2, -ms_new));
+          s[i] = raise ? pv * kFixFactor : pv;
+          rs_raised += s[i];
+        }
+        if (raise) rs = rs_raised;
+      }
+      // rescale of the running O and l: exact, whenever the shift moves
+      float alpha = ex2(ms - ms_new);
+      if (raise != raised) alpha = raise ? alpha * kFixFactor : alpha / kFixFactor;
+      (void)ec;
+      (void)ed;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(s[c * 32 + 2 * i], p.scale_log2, -ms_new));
-          const float p1 = ex2(fmaf(s[c * 32 + 2 * i + 1], p.scale_log2, -ms_new));
-          rs0 += p0;
-          rs1 += p1;
-          pk[i] = pack_bf16(p0, p1);
-        }
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]);
         tmem_st16(t_s + c * 16, pk);
       }
-      l = l * alpha + (rs0 + rs1);
+      l = l * alpha + rs;
       tmem_st_wait();
 
       if (j > 0) {
@@ -276,14 +330,20 @@ __global__ void __launch_bounds__(320, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (j - 1) & 1, wd));
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, ms_new != ms)) {
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+          const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
             tmem_ld32(t_o + c * 32, o);
             tmem_ld_wait(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            for (int i = 0; i < 16; ++i) {
+              float y0, y1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), y0, y1);
+              o[2 * i] = __float_as_uint(y0);
+              o[2 * i + 1] = __float_as_uint(y1);
+            }
             tmem_st32(t_o + c * 32, o);
           }
           tmem_st_wait();
@@ -294,6 +354,7 @@ __global__ void __launch_bounds__(320, 1)
       m = m_new;
       cnt = c_new;
       ms = ms_new;
+      raised = raise;
     }
 
     if (ok && n_t > 0) {
@@ -318,7 +379,7 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         if (row < p.N) {
-          p.lse[size_t(bh) * p.N + row] = (ms + lg2(l)) * kLn2;
+          p.lse[size_t(bh) * p.N + row] = (ms + (raised ? p.delta_log2 : 0.f) + lg2(l)) * kLn2;
           if (p.ties) p.ties[size_t(bh) * p.N + row] = cnt | (ever_repeated ? (1 << 30) : 0);
         }
       }
