@@ -151,7 +151,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   prm.scale_log2 = float(double(scale) * 1.4426950408889634);
   prm.delta_log2 = fix_mode ? float(kDeltaLog2) : 0.f;
   prm.fix = fix_mode;
-  const dim3 grid(unsigned(prm.n_pairs) * unsigned(BH));
+  const int n_items = prm.n_pairs * BH;
+  const dim3 grid(unsigned(n_items < st->num_sms ? n_items : st->num_sms));
   if (d == 64)
     fa_fwd_kernel<64><<<grid, FwdLayout<64>::kThreads, FwdLayout<64>::kAlloc, stream>>>(mq, mk, mv, prm);
   else
@@ -238,7 +239,8 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, c
   prm.causal = causal;
   prm.scale = scale;
   prm.scale_log2 = float(double(scale) * 1.4426950408889634);
-  const dim3 grid(unsigned(prm.n_kv) * unsigned(BH));
+  const int n_items = prm.n_kv * BH;
+  const dim3 grid(unsigned(n_items < st->num_sms ? n_items : st->num_sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
     fa_bwd_kernel<64><<<grid, BwdLayout<64>::kThreads, BwdLayout<64>::kAlloc, s>>>(mq, mk, mv, mdo, mdq, prm);

@@ -88,10 +88,12 @@ struct BwdLayout {
   static constexpr int kSub = D / 64;
   static constexpr int kSubBytes = 128 * 64 * 2;
   static constexpr int kTileBytes = kSub * kSubBytes;
-  static constexpr int kKOff = 0;
-  static constexpr int kVOff = kTileBytes;
-  static constexpr int kDOStages = (D == 64) ? 2 : 1;      // d=128: one dO buffer, refilled after dV
-  static constexpr int kQOff = 2 * kTileBytes;             // 2 stages
+  // d=64 double-buffers K/V so the next item's keys load during this one;
+  // d=128 has no room and keeps one dO buffer, refilled after dV.
+  static constexpr int kKVStages = (D == 64) ? 2 : 1;
+  static constexpr int kDOStages = (D == 64) ? 2 : 1;
+  static constexpr int kKVOff = 0;                          // stage s: K, then V
+  static constexpr int kQOff = kKVStages * 2 * kTileBytes;  // 2 stages
   static constexpr int kDOOff = kQOff + 2 * kTileBytes;
   static constexpr int kDSOff = kDOOff + kDOStages * kTileBytes;   // dS, [128 keys][128 queries] bf16, MN-major
   static constexpr int kStatOff = kDSOff + 2 * kSubBytes;  // 2 stages x (-LSE*log2e, D) x 128 floats
@@ -104,9 +106,9 @@ struct BwdLayout {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 512;
   static constexpr int kLaunchRegs = 128;                  // per thread, fixed by __launch_bounds__(512, 1)
-  static constexpr uint32_t kComputeRegs = 168;
-  static constexpr uint32_t kDrainRegs = 104;
-  static constexpr uint32_t kOtherRegs = 72;
+  static constexpr uint32_t kComputeRegs = 152;
+  static constexpr uint32_t kDrainRegs = 112;
+  static constexpr uint32_t kOtherRegs = 96;
   static_assert(128 * (2 * kComputeRegs + kDrainRegs + kOtherRegs) <= kThreads * kLaunchRegs,
                 "register split exceeds the pool");
   // TMEM columns.  d = 64: P_bar^T has its own 64 columns, so S of the next
@@ -118,21 +120,43 @@ struct BwdLayout {
   static constexpr uint32_t kTmPT = kWide ? 0 : 448;
   // column of P_bar^T / dS^T for MMA K-step k (16 queries = 8 columns): the
   // query half h = k / 4 was written by the warps that own that half
-  __host__ __device__ static constexpr uint32_t pt_col(int k) { return kWide ? kTmS + 64 * (k >> 2) + 8 * (k & 3) : kTmPT + 8 * k; }
+  __host__ __device__ static constexpr uint32_t pt_col(int k) {
+    return kWide ? kTmS + 64 * (k >> 2) + 8 * (k & 3) : kTmPT + 8 * k;
+  }
   __host__ __device__ static constexpr uint32_t dst_col(int k) { return kTmDP + 64 * (k >> 2) + 8 * (k & 3); }
 };
+
+// One work item = one (batch*head, 128-key tile); items are numbered heavy
+// first (causal: the first key tiles are seen by the most query tiles).  CTAs
+// are persistent and sweep the sorted items with snake_item()
+struct BwdItem {
+  int bh, kv_tile, key0, i_start, n_it;
+};
+
+__device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
+  BwdItem w;
+  w.kv_tile = item / p.BH;
+  w.bh = item % p.BH;
+  w.key0 = w.kv_tile * 128;
+  const int n_q = (p.N + 127) / 128;
+  w.i_start = p.causal ? w.kv_tile : 0;
+  w.n_it = n_q - w.i_start;
+  return w;
+}
 
 // Roles (16 warps):
 //   warps 0-7   key-row math; warp w owns keys 32*(w%4).. (TMEM lane quarter
 //               w%4) and queries 64*(w/4).. of each tile: P^T, dS^T
 //   warps 8-11  dQ drain (thread r owns query r; TMA reduce-add of 32 x 32
 //               FP32 boxes staged in shared memory) and the dK/dV epilogue
-//   warp  12    producer: K, V once; Q_i, dO_i (TMA) plus LSE_i, D_i per step
+//   warp  12    producer: K, V per item; Q_i, dO_i (TMA) plus LSE_i, D_i per step
 //   warp  13    TMEM allocator + tcgen05.mma issuer
 //   warps 14-15 idle (complete the fourth warpgroup)
 // MMA order per query tile i (the tensor core runs the next tile's S while
 // the CUDA cores form dS_i, and dK_i, dQ_i, dP_{i+1} while they form P_{i+1}):
 //   dV_i += P_bar_i^T dO_i | S_{i+1} | dK_i += dS_i^T Q_i | dQ_i = dS_i K | dP_{i+1}
+// Barrier phases run on per-CTA counters, so items follow one another without
+// re-initialisation: `g` counts query-tile steps, `n_done` counts items.
 template <int D>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -141,20 +165,23 @@ __global__ void __launch_bounds__(512, 1)
   using L = BwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* kv_full = bars;
-  uint64_t* q_full = bars + 1;    // [2]
-  uint64_t* q_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 6;
-  uint64_t* dp_full = bars + 7;
-  uint64_t* ds_full = bars + 8;
-  uint64_t* dq_full = bars + 9;
-  uint64_t* dq_free = bars + 10;
-  uint64_t* dkv_done = bars + 11;
-  uint64_t* pt_free = bars + 12;
-  uint64_t* do_full = bars + 13;   // [2]
-  uint64_t* do_empty = bars + 15;  // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* kv_full = bars;        // [2]
+  uint64_t* kv_empty = bars + 2;   // [2]
+  uint64_t* q_full = bars + 4;     // [2]
+  uint64_t* q_empty = bars + 6;    // [2]
+  uint64_t* do_full = bars + 8;    // [2]
+  uint64_t* do_empty = bars + 10;  // [2]
+  uint64_t* s_full = bars + 12;
+  uint64_t* p_full = bars + 13;
+  uint64_t* dp_full = bars + 14;
+  uint64_t* ds_full = bars + 15;
+  uint64_t* dq_full = bars + 16;
+  uint64_t* dq_free = bars + 17;
+  uint64_t* dkv_done = bars + 18;
+  uint64_t* dkv_free = bars + 19;
+  uint64_t* pt_free = bars + 20;
+  uint64_t* mma_done = bars + 21;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* stats = reinterpret_cast<float*>(smem + L::kStatOff);   // [stage][-lse2 | dsum][128]
 
@@ -164,20 +191,18 @@ __global__ void __launch_bounds__(512, 1)
     if (threadIdx.x == 0) atomicExch(p.dev_error, kDevErrSmemAlign);
     return;
   }
-  const int kv_tile = int(blockIdx.x) / p.BH;
-  const int bh = int(blockIdx.x) % p.BH;
-  const int key0 = kv_tile * 128;
-  const int n_q = (p.N + 127) / 128;
-  const int i_start = p.causal ? kv_tile : 0;
-  const int n_it = n_q - i_start;
+  const int n_items = p.n_kv * p.BH;
   const int warp = int(warp_id());
   const int lane = int(lane_id());
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
     for (int s = 0; s < 2; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
+      mbar_init(&do_full[s], 1);
+      mbar_init(&do_empty[s], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(p_full, 256);
@@ -186,11 +211,9 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 128);
     mbar_init(dkv_done, 1);
+    mbar_init(dkv_free, 128);
     mbar_init(pt_free, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&do_full[s], 1);
-      mbar_init(&do_empty[s], 1);
-    }
+    mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -218,46 +241,58 @@ __global__ void __launch_bounds__(512, 1)
       // ----------------------------------------------------------- producer
       const uint64_t pol_kv = l2_policy_evict_first();
       const uint64_t pol_q = l2_policy_evict_last();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(kv_full, uint32_t(2 * L::kTileBytes));
-        for (int s = 0; s < L::kSub; ++s) {
-          tma_load_3d(smem + L::kKOff + s * L::kSubBytes, &tm_k, kv_full, s * 64, key0, bh, pol_kv);
-          tma_load_3d(smem + L::kVOff + s * L::kSubBytes, &tm_v, kv_full, s * 64, key0, bh, pol_kv);
-        }
-      }
       const float kLog2e = 1.4426950408889634f;
-      for (int it = 0; it < n_it; ++it) {
-        const int st = it & 1;
-        const int q0 = (i_start + it) * 128;
-        if (!__all_sync(0xffffffffu, mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1, wd))) break;
-        float* nlse = stats + st * 256;
-        float* dd = nlse + 128;
+      uint32_t g = 0;        // query-tile steps loaded
+      uint32_t n_done = 0;   // items started
+      bool ok = true;
+      for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
+        const BwdItem w = bwd_item(p, item);
+        const uint32_t ks = n_done % L::kKVStages;
+        ok = __all_sync(0xffffffffu, mbar_wait(&kv_empty[ks], ((n_done / L::kKVStages) & 1) ^ 1, wd));
+        if (!ok) break;
+        if (lane == 0) {
+          uint8_t* sk = smem + L::kKVOff + ks * 2 * L::kTileBytes;
+          mbar_arrive_expect_tx(&kv_full[ks], uint32_t(2 * L::kTileBytes));
+          for (int s = 0; s < L::kSub; ++s) {
+            tma_load_3d(sk + s * L::kSubBytes, &tm_k, &kv_full[ks], s * 64, w.key0, w.bh, pol_kv);
+            tma_load_3d(sk + L::kTileBytes + s * L::kSubBytes, &tm_v, &kv_full[ks], s * 64, w.key0, w.bh, pol_kv);
+          }
+        }
+        for (int it = 0; it < w.n_it; ++it, ++g) {
+          const uint32_t st = g & 1;
+          const int q0 = (w.i_start + it) * 128;
+          ok = __all_sync(0xffffffffu, mbar_wait(&q_empty[st], ((g >> 1) & 1) ^ 1, wd));
+          if (!ok) break;
+          float* nlse = stats + st * 256;
+          float* dd = nlse + 128;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int r = lane * 4 + u;
-          const int row = q0 + r;
-          const bool in = row < p.N;
-          // rows past N: P = 2^(-inf) = 0 and D = 0, so they add nothing
-          nlse[r] = in ? -p.lse[size_t(bh) * p.N + row] * kLog2e : -__int_as_float(0x7f800000);
-          dd[r] = in ? p.dsum[size_t(bh) * p.N + row] : 0.f;
+          for (int u = 0; u < 4; ++u) {
+            const int r = lane * 4 + u;
+            const int row = q0 + r;
+            const bool in = row < p.N;
+            // rows past N: P = 2^(-inf) = 0 and D = 0, so they add nothing
+            nlse[r] = in ? -p.lse[size_t(w.bh) * p.N + row] * kLog2e : -__int_as_float(0x7f800000);
+            dd[r] = in ? p.dsum[size_t(w.bh) * p.N + row] : 0.f;
+          }
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&q_full[st], uint32_t(L::kTileBytes));
+            for (int s = 0; s < L::kSub; ++s)
+              tma_load_3d(smem + L::kQOff + st * L::kTileBytes + s * L::kSubBytes, &tm_q, &q_full[st], s * 64, q0,
+                          w.bh, pol_q);
+          }
+          // dO_i: with a single buffer it is refilled once dV_{i-1} has read it
+          const uint32_t sd = g % L::kDOStages;
+          ok = __all_sync(0xffffffffu, mbar_wait(&do_empty[sd], ((g / L::kDOStages) & 1) ^ 1, wd));
+          if (!ok) break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&do_full[sd], uint32_t(L::kTileBytes));
+            for (int s = 0; s < L::kSub; ++s)
+              tma_load_3d(smem + L::kDOOff + sd * L::kTileBytes + s * L::kSubBytes, &tm_do, &do_full[sd], s * 64,
+                          q0, w.bh, pol_q);
+          }
+          __syncwarp();
         }
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&q_full[st], uint32_t(L::kTileBytes));
-          for (int s = 0; s < L::kSub; ++s)
-            tma_load_3d(smem + L::kQOff + st * L::kTileBytes + s * L::kSubBytes, &tm_q, &q_full[st], s * 64, q0,
-                        bh, pol_q);
-        }
-        // dO_i: with a single buffer it is refilled once dV_{i-1} has read it
-        const int sd = it % L::kDOStages;
-        if (!__all_sync(0xffffffffu, mbar_wait(&do_empty[sd], ((it / L::kDOStages) & 1) ^ 1, wd))) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&do_full[sd], uint32_t(L::kTileBytes));
-          for (int s = 0; s < L::kSub; ++s)
-            tma_load_3d(smem + L::kDOOff + sd * L::kTileBytes + s * L::kSubBytes, &tm_do, &do_full[sd], s * 64, q0,
-                        bh, pol_q);
-        }
-        __syncwarp();
       }
     } else if (warp == 13) {
       // ---------------------------------------------------------- MMA issuer
@@ -265,8 +300,6 @@ __global__ void __launch_bounds__(512, 1)
         constexpr uint32_t kIdS = make_idesc_bf16(128, 128, 0, 0);   // K Q^T, V dO^T: K-major operands
         constexpr uint32_t kIdAcc = make_idesc_bf16(128, D, 0, 1);   // TMEM A x MN-major B (dV, dK)
         constexpr uint32_t kIdDQ = make_idesc_bf16(128, D, 1, 1);    // dS (MN-major) x K (MN-major)
-        const uint32_t sk = smem_u32(smem + L::kKOff);
-        const uint32_t sv = smem_u32(smem + L::kVOff);
         const uint32_t sds = smem_u32(smem + L::kDSOff);
         auto kmajor_mma = [&](uint32_t d_tm, uint32_t a, uint32_t b) {
 #pragma unroll
@@ -275,65 +308,84 @@ __global__ void __launch_bounds__(512, 1)
             umma_ss(d_tm, make_sdesc_sw128(a + off, 16, 1024), make_sdesc_sw128(b + off, 16, 1024), kIdS, k > 0);
           }
         };
-        auto q_of = [&](int it) { return smem_u32(smem + L::kQOff + (it & 1) * L::kTileBytes); };
-        auto do_of = [&](int it) { return smem_u32(smem + L::kDOOff + (it % L::kDOStages) * L::kTileBytes); };
-        auto wait_do = [&](int it) {
-          return mbar_wait(&do_full[it % L::kDOStages], (it / L::kDOStages) & 1, wd);
+        auto q_of = [&](uint32_t gg) { return smem_u32(smem + L::kQOff + (gg & 1) * L::kTileBytes); };
+        auto do_of = [&](uint32_t gg) {
+          return smem_u32(smem + L::kDOOff + (gg % L::kDOStages) * L::kTileBytes);
         };
-        bool ok = mbar_wait(kv_full, 0, wd) && mbar_wait(&q_full[0], 0, wd) && wait_do(0);
-        if (ok) {
+        auto wait_q = [&](uint32_t gg) { return mbar_wait(&q_full[gg & 1], (gg >> 1) & 1, wd); };
+        auto wait_do = [&](uint32_t gg) {
+          return mbar_wait(&do_full[gg % L::kDOStages], (gg / L::kDOStages) & 1, wd);
+        };
+        uint32_t g = 0;        // query-tile steps issued
+        uint32_t n_done = 0;   // items started
+        bool ok = true;
+        for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
+          const BwdItem w = bwd_item(p, item);
+          const uint32_t ks = n_done % L::kKVStages;
+          const uint32_t sk = smem_u32(smem + L::kKVOff + ks * 2 * L::kTileBytes);
+          const uint32_t sv = sk + L::kTileBytes;
+          if (!(ok = mbar_wait(&kv_full[ks], (n_done / L::kKVStages) & 1, wd) && wait_q(g) && wait_do(g))) break;
           tc_fence_after();
-          kmajor_mma(tmem + L::kTmS, sk, q_of(0));     // S^T_0 = K Q_0^T
+          kmajor_mma(tmem + L::kTmS, sk, q_of(g));     // S^T = K Q^T of the item's first query tile
           umma_commit(s_full);
-          kmajor_mma(tmem + L::kTmDP, sv, do_of(0));   // dP^T_0 = V dO_0^T
+          if (L::kWide && g > 0) {                      // the previous dQ shares the dP^T columns
+            if (!(ok = mbar_wait(dq_free, (g - 1) & 1, wd))) break;
+            tc_fence_after();
+          }
+          kmajor_mma(tmem + L::kTmDP, sv, do_of(g));   // dP^T = V dO^T
           umma_commit(dp_full);
-        }
-        for (int it = 0; ok && it < n_it; ++it) {
-          const uint32_t sq = q_of(it);
-          const uint32_t sdo = do_of(it);
-          if (!(ok = mbar_wait(p_full, it & 1, wd))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < 8; ++k)                   // dV += P_bar^T dO_i
-            umma_ts(tmem + L::kTmDV, tmem + L::pt_col(k), make_sdesc_sw128(sdo + k * 2048, L::kSubBytes, 1024),
-                    kIdAcc, (it > 0 || k > 0) ? 1u : 0u);
-          umma_commit(pt_free);
-          umma_commit(&do_empty[it % L::kDOStages]);    // dP_i and dV_i were the readers of dO_i
-          if (it + 1 < n_it) {                          // S^T_{i+1}
-            if (!(ok = mbar_wait(&q_full[(it + 1) & 1], ((it + 1) >> 1) & 1, wd))) break;
+          // the first dV/dK MMA of an item overwrites the accumulators: the
+          // previous item's epilogue must have read them
+          if (!(ok = mbar_wait(dkv_free, (n_done & 1) ^ 1, wd))) break;
+          for (int it = 0; ok && it < w.n_it; ++it, ++g) {
+            const uint32_t sq = q_of(g);
+            const uint32_t sdo = do_of(g);
+            if (!(ok = mbar_wait(p_full, g & 1, wd))) break;
             tc_fence_after();
-            kmajor_mma(tmem + L::kTmS, sk, q_of(it + 1));
-            umma_commit(s_full);
-          }
-          if (!(ok = mbar_wait(ds_full, it & 1, wd))) break;
-          tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < 8; ++k)                   // dK += dS^T Q_i
-            umma_ts(tmem + L::kTmDK, tmem + L::dst_col(k), make_sdesc_sw128(sq + k * 2048, L::kSubBytes, 1024),
-                    kIdAcc, (it > 0 || k > 0) ? 1u : 0u);
-          if (!L::kWide && it > 0) {                    // the drain has read dQ_{i-1}
-            if (!(ok = mbar_wait(dq_free, (it - 1) & 1, wd))) break;
+            for (int k = 0; k < 8; ++k)                 // dV += P_bar^T dO_i
+              umma_ts(tmem + L::kTmDV, tmem + L::pt_col(k), make_sdesc_sw128(sdo + k * 2048, L::kSubBytes, 1024),
+                      kIdAcc, (it > 0 || k > 0) ? 1u : 0u);
+            umma_commit(pt_free);
+            umma_commit(&do_empty[g % L::kDOStages]);   // dP_i and dV_i were the readers of dO_i
+            if (it + 1 < w.n_it) {                      // S^T_{i+1}
+              if (!(ok = wait_q(g + 1))) break;
+              tc_fence_after();
+              kmajor_mma(tmem + L::kTmS, sk, q_of(g + 1));
+              umma_commit(s_full);
+            }
+            if (!(ok = mbar_wait(ds_full, g & 1, wd))) break;
             tc_fence_after();
-          }
 #pragma unroll
-          for (int k = 0; k < 8; ++k)                   // dQ_i = dS K
-            umma_ss(tmem + L::kTmDQ, make_sdesc_sw128(sds + k * 2048, L::kSubBytes, 1024),
-                    make_sdesc_sw128(sk + k * 2048, L::kSubBytes, 1024), kIdDQ, k > 0 ? 1u : 0u);
-          umma_commit(dq_full);
-          umma_commit(&q_empty[it & 1]);
-          if (it + 1 < n_it) {                          // dP^T_{i+1}
-            if (L::kWide) {                             // dQ_i shares the dP^T columns
-              if (!(ok = mbar_wait(dq_free, it & 1, wd))) break;
+            for (int k = 0; k < 8; ++k)                 // dK += dS^T Q_i
+              umma_ts(tmem + L::kTmDK, tmem + L::dst_col(k), make_sdesc_sw128(sq + k * 2048, L::kSubBytes, 1024),
+                      kIdAcc, (it > 0 || k > 0) ? 1u : 0u);
+            if (!L::kWide && g > 0) {                   // the drain has read dQ of the previous step
+              if (!(ok = mbar_wait(dq_free, (g - 1) & 1, wd))) break;
               tc_fence_after();
             }
-            if (!(ok = wait_do(it + 1))) break;
-            tc_fence_after();
-            kmajor_mma(tmem + L::kTmDP, sv, do_of(it + 1));
-            umma_commit(dp_full);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)                 // dQ_i = dS K
+              umma_ss(tmem + L::kTmDQ, make_sdesc_sw128(sds + k * 2048, L::kSubBytes, 1024),
+                      make_sdesc_sw128(sk + k * 2048, L::kSubBytes, 1024), kIdDQ, k > 0 ? 1u : 0u);
+            umma_commit(dq_full);
+            umma_commit(&q_empty[g & 1]);
+            if (it + 1 < w.n_it) {                      // dP^T_{i+1}
+              if (L::kWide) {                           // dQ_i shares the dP^T columns
+                if (!(ok = mbar_wait(dq_free, g & 1, wd))) break;
+                tc_fence_after();
+              }
+              if (!(ok = wait_do(g + 1))) break;
+              tc_fence_after();
+              kmajor_mma(tmem + L::kTmDP, sv, do_of(g + 1));
+              umma_commit(dp_full);
+            }
           }
+          umma_commit(&kv_empty[ks]);                   // K and V of this item are no longer read
+          umma_commit(dkv_done);                        // dK, dV of this item are final
         }
-        umma_commit(dkv_done);
-        mbar_wait(dkv_done, 0, wd);
+        umma_commit(mma_done);
+        mbar_wait(mma_done, 0, wd);
       }
       __syncwarp();
     }
@@ -343,106 +395,111 @@ __global__ void __launch_bounds__(512, 1)
     const int quarter = warp & 3;
     const int half = warp >> 2;                      // queries 64*half .. +63
     const int kr = quarter * 32 + lane;              // key within the tile
-    const int key = key0 + kr;
-    const bool key_in = key < p.N;
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     const uint32_t t_s = tmem + lane_base + L::kTmS + 64 * half;
     const uint32_t t_dp = tmem + lane_base + L::kTmDP + 64 * half;
     const uint32_t t_pt = tmem + lane_base + (L::kWide ? L::kTmS + 64 * half : L::kTmPT + 32 * half);
     uint8_t* ds_row = smem + L::kDSOff + half * L::kSubBytes + kr * 128;
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
-    for (int it = 0; it < n_it; ++it) {
-      const int st = it & 1;
-      const int qt = i_start + it;
-      const float* nlse = stats + st * 256 + 64 * half;
-      const float* dd = stats + st * 256 + 128 + 64 * half;
-      // q_full publishes this stage's LSE/D (written by the producer's lanes)
-      if (!__all_sync(0xffffffffu, mbar_wait(&q_full[st], (it >> 1) & 1, wd))) break;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full, it & 1, wd))) break;
-      tc_fence_after();
-      // P^T: P[q] = 2^(S*scale_log2 - LSE2[q]); masked entries are 0
-      uint32_t pk[32];
-      {
-        uint32_t r[2][32];
-        tmem_ld32(t_s, r[0]);
-        tmem_ld32(t_s + 32, r[1]);
-        tmem_ld_wait(r[0]);
-        tmem_ld_wait(r[1]);
-        const bool diag = p.causal && qt == kv_tile;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int q = 2 * i;                         // query within this half
-          const uint64_t nl = *reinterpret_cast<const uint64_t*>(nlse + q);
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
-                                   __uint_as_float(r[i >> 4][(2 * i + 1) & 31])), c2, nl), x0, x1);
-          float p0 = ex2(x0), p1 = ex2(x1);
-          const int qg = 64 * half + q;                // query within the tile
-          if (!key_in || (diag && qg < kr)) p0 = 0.f;
-          if (!key_in || (diag && qg + 1 < kr)) p1 = 0.f;
-          pk[i] = pack_bf16(p0, p1);
-        }
-      }
-      if (!L::kWide && it > 0) {                       // dV_{i-1} has read P_bar^T_{i-1}
-        if (!__all_sync(0xffffffffu, mbar_wait(pt_free, (it - 1) & 1, wd))) break;
+    uint32_t g = 0;
+    bool ok = true;
+    for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd)) {
+      const BwdItem w = bwd_item(p, item);
+      const bool key_in = w.key0 + kr < p.N;
+      for (int it = 0; it < w.n_it; ++it, ++g) {
+        const uint32_t st = g & 1;
+        const int qt = w.i_start + it;
+        const float* nlse = stats + st * 256 + 64 * half;
+        const float* dd = stats + st * 256 + 128 + 64 * half;
+        // q_full publishes this stage's LSE/D (written by the producer's lanes)
+        ok = __all_sync(0xffffffffu, mbar_wait(&q_full[st], (g >> 1) & 1, wd)) &&
+             __all_sync(0xffffffffu, mbar_wait(s_full, g & 1, wd));
+        if (!ok) break;
         tc_fence_after();
-      }
-      {
-        uint32_t w[16];
+        // P^T: P[q] = 2^(S*scale_log2 - LSE2[q]); masked entries are 0
+        uint32_t pk[32];
+        {
+          uint32_t r[2][32];
+          tmem_ld32(t_s, r[0]);
+          tmem_ld32(t_s + 32, r[1]);
+          tmem_ld_wait(r[0]);
+          tmem_ld_wait(r[1]);
+          const bool diag = p.causal && qt == w.kv_tile;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = pk[i];
-        tmem_st16(t_pt, w);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = pk[16 + i];
-        tmem_st16(t_pt + 16, w);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(p_full);
-
-      if (!__all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, wd))) break;
-      tc_fence_after();
-      // dS^T = P_bar * (dP - D[q])
-      uint32_t dsw[32];
-      {
-        uint32_t r[2][32];
-        tmem_ld32(t_dp, r[0]);
-        tmem_ld32(t_dp + 32, r[1]);
-        tmem_ld_wait(r[0]);
-        tmem_ld_wait(r[1]);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[i]));
-          const uint64_t dq2 = *reinterpret_cast<const uint64_t*>(dd + 2 * i);
-          const uint64_t dp2 = f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
-                                       __uint_as_float(r[i >> 4][(2 * i + 1) & 31]));
-          float y0, y1;
-          f2_unpack(f2_mul(f2_fma(dq2, f2_pack(-1.f, -1.f), dp2), f2_pack(pp.x, pp.y)), y0, y1);
-          dsw[i] = pack_bf16(y0, y1);
+          for (int i = 0; i < 32; ++i) {
+            const int q = 2 * i;                       // query within this half
+            const uint64_t nl = *reinterpret_cast<const uint64_t*>(nlse + q);
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
+                                     __uint_as_float(r[i >> 4][(2 * i + 1) & 31])), c2, nl), x0, x1);
+            float p0 = ex2(x0), p1 = ex2(x1);
+            const int qg = 64 * half + q;              // query within the tile
+            if (!key_in || (diag && qg < kr)) p0 = 0.f;
+            if (!key_in || (diag && qg + 1 < kr)) p1 = 0.f;
+            pk[i] = pack_bf16(p0, p1);
+          }
         }
-      }
-      {
-        uint32_t w[16];
+        if (!L::kWide && g > 0) {                      // dV of the previous step has read P_bar^T
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(pt_free, (g - 1) & 1, wd)))) break;
+          tc_fence_after();
+        }
+        {
+          uint32_t wv[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = dsw[i];
-        tmem_st16(t_dp, w);
+          for (int i = 0; i < 16; ++i) wv[i] = pk[i];
+          tmem_st16(t_pt, wv);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = dsw[16 + i];
-        tmem_st16(t_dp + 16, w);
-      }
-      // dS into shared memory for dQ = dS K: MN-major, 128-byte swizzle
-      if (it > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (it - 1) & 1, wd))) break;
-      }
+          for (int i = 0; i < 16; ++i) wv[i] = pk[16 + i];
+          tmem_st16(t_pt + 16, wv);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(p_full);
+
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(dp_full, g & 1, wd)))) break;
+        tc_fence_after();
+        // dS^T = P_bar * (dP - D[q])
+        uint32_t dsw[32];
+        {
+          uint32_t r[2][32];
+          tmem_ld32(t_dp, r[0]);
+          tmem_ld32(t_dp + 32, r[1]);
+          tmem_ld_wait(r[0]);
+          tmem_ld_wait(r[1]);
 #pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16) {
-        uint4* dst = reinterpret_cast<uint4*>(ds_row + ((c16 ^ (kr & 7)) << 4));
-        *dst = make_uint4(dsw[c16 * 4], dsw[c16 * 4 + 1], dsw[c16 * 4 + 2], dsw[c16 * 4 + 3]);
+          for (int i = 0; i < 32; ++i) {
+            const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[i]));
+            const uint64_t dq2 = *reinterpret_cast<const uint64_t*>(dd + 2 * i);
+            const uint64_t dp2 = f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
+                                         __uint_as_float(r[i >> 4][(2 * i + 1) & 31]));
+            float y0, y1;
+            f2_unpack(f2_mul(f2_fma(dq2, f2_pack(-1.f, -1.f), dp2), f2_pack(pp.x, pp.y)), y0, y1);
+            dsw[i] = pack_bf16(y0, y1);
+          }
+        }
+        {
+          uint32_t wv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) wv[i] = dsw[i];
+          tmem_st16(t_dp, wv);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) wv[i] = dsw[16 + i];
+          tmem_st16(t_dp + 16, wv);
+        }
+        // dS into shared memory for dQ = dS K: MN-major, 128-byte swizzle
+        if (g > 0) {                                   // dQ of the previous step has read it
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_full, (g - 1) & 1, wd)))) break;
+        }
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) {
+          uint4* dst = reinterpret_cast<uint4*>(ds_row + ((c16 ^ (kr & 7)) << 4));
+          *dst = make_uint4(dsw[c16 * 4], dsw[c16 * 4 + 1], dsw[c16 * 4 + 2], dsw[c16 * 4 + 3]);
+        }
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(ds_full);
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(ds_full);
     }
   } else {
     regs_decrease<L::kDrainRegs>();
@@ -453,64 +510,75 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t t_dq = tmem + lane_base + L::kTmDQ;
     uint8_t* stage = smem + L::kDQStageOff + wq * 2 * L::kStageBox;
     uint32_t box_seq = 0;
+    uint32_t g = 0;
+    uint32_t n_done = 0;
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, wd));
+    for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
+      const BwdItem w = bwd_item(p, item);
+      for (int it = 0; it < w.n_it; ++it, ++g) {
+        ok = __all_sync(0xffffffffu, mbar_wait(dq_full, g & 1, wd));
+        if (!ok) break;
+        tc_fence_after();
+        // TMEM -> swizzled 32 x 32 FP32 box in shared memory -> TMA reduce-add
+        // into the FP32 accumulator (rows past N are dropped by the TMA unit)
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(t_dq + c * 32, r);
+          tmem_ld_wait(r);
+          if (c == D / 32 - 1) {                       // dQ is in registers: its TMEM may be reused
+            tc_fence_before();
+            mbar_arrive(dq_free);
+          }
+          uint8_t* box = stage + (box_seq & 1) * L::kStageBox;
+          if (lane == 0) bulk_wait_read<1>();          // the reduce issued from this box is done reading
+          __syncwarp();
+#pragma unroll
+          for (int c16 = 0; c16 < 8; ++c16)
+            *reinterpret_cast<uint4*>(box + lane * 128 + ((c16 ^ (lane & 7)) << 4)) =
+                make_uint4(r[4 * c16], r[4 * c16 + 1], r[4 * c16 + 2], r[4 * c16 + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_3d(&tm_dq, box, c * 32, (w.i_start + it) * 128 + wq * 32, w.bh);
+            bulk_commit();
+          }
+          ++box_seq;
+        }
+      }
+      if (!ok) break;
+      // epilogue: dV and scale * dK of this item's keys, bf16
+      ok = __all_sync(0xffffffffu, mbar_wait(dkv_done, n_done & 1, wd));
       if (!ok) break;
       tc_fence_after();
-      // TMEM -> swizzled 32 x 32 FP32 box in shared memory -> TMA reduce-add
-      // into the FP32 accumulator (rows past N are dropped by the TMA unit)
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_dq + c * 32, r);
-        tmem_ld_wait(r);
-        uint8_t* box = stage + (box_seq & 1) * L::kStageBox;
-        if (lane == 0) bulk_wait_read<1>();              // the reduce issued from this box is done reading
-        __syncwarp();
-#pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16)
-          *reinterpret_cast<uint4*>(box + lane * 128 + ((c16 ^ (lane & 7)) << 4)) =
-              make_uint4(r[4 * c16], r[4 * c16 + 1], r[4 * c16 + 2], r[4 * c16 + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_reduce_add_3d(&tm_dq, box, c * 32, (i_start + it) * 128 + wq * 32, bh);
-          bulk_commit();
-        }
-        ++box_seq;
-      }
-      tc_fence_before();
-      mbar_arrive(dq_free);
-    }
-    if (lane == 0) bulk_wait<0>();                      // every reduce-add has landed
-    __syncwarp();
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dkv_done, 0, wd));
-    if (ok) {
-      tc_fence_after();
-      const int key = key0 + rr;
+      const int key = w.key0 + rr;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t t_src = tmem + lane_base + (which ? L::kTmDK : L::kTmDV);
         const float mul = which ? p.scale : 1.f;
-        __nv_bfloat16* out = (which ? p.dk : p.dv) + (size_t(bh) * p.N + key) * D;
+        uint32_t ov[D / 2];
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
           tmem_ld32(t_src + c * 32, r);
           tmem_ld_wait(r);
-          uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            w[i] = pack_bf16(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
-          if (key < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+            ov[c * 16 + i] = pack_bf16(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
+        }
+        if (which == 1) {
+          tc_fence_before();
+          mbar_arrive(dkv_free);                     // the next item may overwrite dK, dV
+        }
+        if (key < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>((which ? p.dk : p.dv) + (size_t(w.bh) * p.N + key) * D);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-          }
+          for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
         }
       }
     }
+    if (lane == 0) bulk_wait<0>();                     // every reduce-add has landed
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -9,17 +9,18 @@
 // the row maximum of S occurs more than once, raise the shift m so every
 // exponent, the maxima included, is strictly below 1.
 //
-// One CTA = one (batch, head) and two 128-row query tiles, processed in
-// ping-pong so the tensor core works on one tile while the other tile's
-// softmax runs on the CUDA cores:
+// Persistent CTAs (one per SM) loop over work items; one item = one
+// (batch, head) and two 128-row query tiles, processed in ping-pong so the
+// tensor core works on one tile while the other tile's softmax runs on the
+// CUDA cores.  An item's epilogue overlaps the next item's first MMAs:
 //   warps 0-3  softmax of query tile 0 (thread r owns row r: TMEM lane r)
 //   warps 4-7  softmax of query tile 1
 //   warp  8    TMA producer: Q tiles once, then a ring of K/V stages
 //   warp  9    TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 10-11 idle (they complete the third warpgroup)
 // Registers: launched at 168 per thread (384 threads); the third warpgroup
-// gives back down to 56 and the two softmax warpgroups take 224 each:
-// 128 * (224 + 224 + 56) = 384 * 168.
+// gives back down to 88 and the two softmax warpgroups take 208 each:
+// 128 * (208 + 208 + 88) = 384 * 168.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 after.
 // P_bar (bf16, two per 32-bit column) overwrites the first 64 columns of S_t
 // and is the A operand of O_t += P_bar V (V is the MN-major B operand).
@@ -54,10 +55,29 @@ struct FwdLayout {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 384;
   static constexpr int kLaunchRegs = 168;       // per thread, fixed by __launch_bounds__(384, 1)
-  static constexpr uint32_t kSoftmaxRegs = 224;
-  static constexpr uint32_t kOtherRegs = 56;
+  static constexpr uint32_t kSoftmaxRegs = 208;
+  static constexpr uint32_t kOtherRegs = 88;
   static_assert(128 * (2 * kSoftmaxRegs + kOtherRegs) <= kThreads * kLaunchRegs, "register split exceeds the pool");
 };
+
+// One work item = one (batch*head, pair of query tiles).  Items are numbered
+// heavy first (causal: the last query tiles see the most keys); the CTAs are
+// persistent and sweep the sorted items with snake_item()
+struct FwdItem {
+  int bh, q0_row, n0, n1, nmax;
+};
+
+__device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
+  FwdItem it;
+  const int pair = p.causal ? (p.n_pairs - 1 - item / p.BH) : item / p.BH;
+  it.bh = item % p.BH;
+  it.q0_row = pair * 256;
+  const int n_kv = (p.N + 127) / 128;
+  it.n0 = p.causal ? min(2 * pair + 1, n_kv) : n_kv;
+  it.n1 = (it.q0_row + 128 < p.N) ? (p.causal ? min(2 * pair + 2, n_kv) : n_kv) : 0;
+  it.nmax = max(it.n0, it.n1);
+  return it;
+}
 
 template <int D>
 __global__ void __launch_bounds__(384, 1)
@@ -71,30 +91,24 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;
   uint64_t* kv_empty = kv_full + L::kStages;
   uint64_t* s_full = kv_empty + L::kStages;  // [2]
   uint64_t* p_full = s_full + 2;             // [2]
   uint64_t* o_done = p_full + 2;             // [2]
-  uint64_t* mma_done = o_done + 2;
+  uint64_t* o_free = o_done + 2;             // [2]
+  uint64_t* mma_done = o_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  // Causal tiles get heavier with the query index: launch the heavy ones first.
-  const int pair = p.causal ? (p.n_pairs - 1 - int(blockIdx.x) / p.BH) : int(blockIdx.x) / p.BH;
-  const int bh = int(blockIdx.x) % p.BH;
-  const int q0_row = pair * 256;
-  const int q1_row = q0_row + 128;
-  const int n_kv = (p.N + 127) / 128;
-  const int n0 = p.causal ? min(2 * pair + 1, n_kv) : n_kv;
-  const int n1 = (q1_row < p.N) ? (p.causal ? min(2 * pair + 2, n_kv) : n_kv) : 0;
-  const int nmax = max(n0, n1);
-
+  const int n_items = p.n_pairs * p.BH;
   const int warp = int(warp_id());
   const int lane = int(lane_id());
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
@@ -103,6 +117,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 128);
       mbar_init(&o_done[t], 1);
+      mbar_init(&o_free[t], 128);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -131,77 +146,103 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) {
         const uint64_t pol_q = l2_policy_evict_first();
         const uint64_t pol_kv = l2_policy_evict_last();
-        const int nq = (n1 > 0) ? 2 : 1;
-        mbar_arrive_expect_tx(q_full, uint32_t(nq * L::kTileBytes));
-        for (int t = 0; t < nq; ++t)
-          for (int s = 0; s < L::kSub; ++s)
-            tma_load_3d(smem + L::kQOff + t * L::kTileBytes + s * L::kSubBytes, &tm_q, q_full, s * 64,
-                        q0_row + t * 128, bh, pol_q);
-        for (int j = 0; j < nmax; ++j) {
-          const int st = j % L::kStages;
-          if (!mbar_wait(&kv_empty[st], ((j / L::kStages) & 1) ^ 1, wd)) break;
-          mbar_arrive_expect_tx(&kv_full[st], uint32_t(2 * L::kTileBytes));
-          uint8_t* sk = smem + L::kKVOff + st * 2 * L::kTileBytes;
-          uint8_t* sv = sk + L::kTileBytes;
-          for (int s = 0; s < L::kSub; ++s) {
-            tma_load_3d(sk + s * L::kSubBytes, &tm_k, &kv_full[st], s * 64, j * 128, bh, pol_kv);
-            tma_load_3d(sv + s * L::kSubBytes, &tm_v, &kv_full[st], s * 64, j * 128, bh, pol_kv);
+        uint32_t kv_cnt = 0;   // K/V tiles loaded so far by this CTA
+        uint32_t n_done = 0;   // items started
+        bool ok = true;
+        for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
+          const FwdItem w = fwd_item(p, item);
+          // the previous item's S MMAs must be done with Q
+          if (!(ok = mbar_wait(q_empty, (n_done & 1) ^ 1, wd))) break;
+          const int nq = (w.n1 > 0) ? 2 : 1;
+          mbar_arrive_expect_tx(q_full, uint32_t(nq * L::kTileBytes));
+          for (int t = 0; t < nq; ++t)
+            for (int s = 0; s < L::kSub; ++s)
+              tma_load_3d(smem + L::kQOff + t * L::kTileBytes + s * L::kSubBytes, &tm_q, q_full, s * 64,
+                          w.q0_row + t * 128, w.bh, pol_q);
+          for (int j = 0; j < w.nmax; ++j, ++kv_cnt) {
+            const uint32_t st = kv_cnt % L::kStages;
+            if (!(ok = mbar_wait(&kv_empty[st], ((kv_cnt / L::kStages) & 1) ^ 1, wd))) break;
+            mbar_arrive_expect_tx(&kv_full[st], uint32_t(2 * L::kTileBytes));
+            uint8_t* sk = smem + L::kKVOff + st * 2 * L::kTileBytes;
+            uint8_t* sv = sk + L::kTileBytes;
+            for (int s = 0; s < L::kSub; ++s) {
+              tma_load_3d(sk + s * L::kSubBytes, &tm_k, &kv_full[st], s * 64, j * 128, w.bh, pol_kv);
+              tma_load_3d(sv + s * L::kSubBytes, &tm_v, &kv_full[st], s * 64, j * 128, w.bh, pol_kv);
+            }
           }
         }
       }
     } else if (warp == 9) {
-      // ------------------------------------------------------------ MMA issuer
+      // ---------------------------------------------------------- MMA issuer
       if (lane == 0) {
         constexpr uint32_t kIdS = make_idesc_bf16(128, 128, 0, 0);   // Q K^T: both K-major
         constexpr uint32_t kIdPV = make_idesc_bf16(128, D, 0, 1);    // P_bar V: V is MN-major
         const uint32_t sq = smem_u32(smem + L::kQOff);
         const uint32_t skv = smem_u32(smem + L::kKVOff);
-        auto issue_s = [&](int t, int st) {
+        auto issue_s = [&](int t, uint32_t st) {
           const uint32_t qa = sq + t * L::kTileBytes;
           const uint32_t ka = skv + st * 2 * L::kTileBytes;
-  #pragma unroll
+#pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t off = (k >> 2) * L::kSubBytes + (k & 3) * 32;
             umma_ss(tmem + t * 128, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
                     kIdS, k > 0);
           }
+          umma_commit(&s_full[t]);
         };
-        auto issue_pv = [&](int t, int st, int j) {
+        auto issue_pv = [&](int t, uint32_t st, int j) {
           const uint32_t va = skv + st * 2 * L::kTileBytes + L::kTileBytes;
-  #pragma unroll
+#pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts(tmem + 256 + t * D, tmem + t * 128 + k * 8, make_sdesc_sw128(va + k * 2048, L::kSubBytes, 1024),
-                    kIdPV, (j > 0 || k > 0) ? 1u : 0u);
+            umma_ts(tmem + 256 + t * D, tmem + t * 128 + k * 8,
+                    make_sdesc_sw128(va + k * 2048, L::kSubBytes, 1024), kIdPV, (j > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&o_done[t]);
         };
-        bool ok = mbar_wait(q_full, 0, wd) && mbar_wait(&kv_full[0], 0, wd);
-        if (ok) {
+        uint32_t kv_cnt = 0;           // K/V tiles consumed
+        uint32_t it_cnt[2] = {0, 0};   // softmax iterations per query tile
+        uint32_t ep_cnt[2] = {0, 0};   // items finished per query tile (epilogues)
+        uint32_t n_done = 0;
+        bool ok = true;
+        for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
+          const FwdItem w = fwd_item(p, item);
+          const int nt[2] = {w.n0, w.n1};
+          if (!(ok = mbar_wait(q_full, n_done & 1, wd) &&
+                     mbar_wait(&kv_full[kv_cnt % L::kStages], (kv_cnt / L::kStages) & 1, wd)))
+            break;
           tc_fence_after();
-          if (n0 > 0) { issue_s(0, 0); umma_commit(&s_full[0]); }
-          if (n1 > 0) { issue_s(1, 0); umma_commit(&s_full[1]); }
-        }
-        for (int j = 0; ok && j < nmax; ++j) {
-          const int st = j % L::kStages;
-          const int jn = j + 1;
-          const int stn = jn % L::kStages;
-          if (j < n0) {
-            if (!(ok = mbar_wait(&p_full[0], j & 1, wd))) break;
-            tc_fence_after();
-            issue_pv(0, st, j);
-            umma_commit(&o_done[0]);
+          for (int t = 0; t < 2; ++t)
+            if (nt[t] > 0) issue_s(t, kv_cnt % L::kStages);
+          if (w.nmax == 1) umma_commit(q_empty);
+          for (int j = 0; ok && j < w.nmax; ++j) {
+            const uint32_t st = (kv_cnt + j) % L::kStages;
+            const uint32_t stn = (kv_cnt + j + 1) % L::kStages;
+            for (int t = 0; t < 2; ++t) {
+              if (j < nt[t]) {
+                if (!(ok = mbar_wait(&p_full[t], (it_cnt[t] + j) & 1, wd))) break;
+                // the first P_bar V of an item overwrites O_t: the previous
+                // item's epilogue must have read it
+                if (j == 0 && !(ok = mbar_wait(&o_free[t], (ep_cnt[t] & 1) ^ 1, wd))) break;
+                tc_fence_after();
+                issue_pv(t, st, j);
+              }
+              if (t == 0 && j + 1 < w.nmax) {
+                const uint32_t nxt = kv_cnt + j + 1;
+                if (!(ok = mbar_wait(&kv_full[stn], (nxt / L::kStages) & 1, wd))) break;
+                tc_fence_after();
+                if (j + 1 < nt[0]) issue_s(0, stn);
+              }
+              if (t == 1) {
+                umma_commit(&kv_empty[st]);
+                if (j + 1 < nt[1]) issue_s(1, stn);
+                if (j + 2 == w.nmax) umma_commit(q_empty);   // the item's last S MMAs are issued
+              }
+            }
           }
-          if (jn < nmax) {
-            if (!(ok = mbar_wait(&kv_full[stn], (jn / L::kStages) & 1, wd))) break;
-            tc_fence_after();
+          kv_cnt += w.nmax;
+          for (int t = 0; t < 2; ++t) {
+            it_cnt[t] += nt[t];
+            ep_cnt[t] += (nt[t] > 0) ? 1 : 0;
           }
-          if (jn < n0) { issue_s(0, stn); umma_commit(&s_full[0]); }
-          if (j < n1) {
-            if (!(ok = mbar_wait(&p_full[1], j & 1, wd))) break;
-            tc_fence_after();
-            issue_pv(1, st, j);
-            umma_commit(&o_done[1]);
-          }
-          umma_commit(&kv_empty[st]);
-          if (jn < n1) { issue_s(1, stn); umma_commit(&s_full[1]); }
         }
         // Every MMA must be finished before TMEM is released.
         umma_commit(mma_done);
@@ -213,176 +254,179 @@ __global__ void __launch_bounds__(384, 1)
     regs_increase<L::kSoftmaxRegs>();
     // --------------------------------------------------- softmax warpgroups
     const int t = warp >> 2;
-    const int n_t = t ? n1 : n0;
-    const int row = (t ? q1_row : q0_row) + (warp & 3) * 32 + lane;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t t_s = tmem + lane_base + uint32_t(t * 128);
     const uint32_t t_o = tmem + lane_base + uint32_t(256 + t * D);
-    const int limit = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
     const float sl2 = p.scale_log2;
     // 2^-delta: on a repeated-max row P is computed with the plain shift and
     // then multiplied by this, which is the same as raising m by delta; each
     // maximum lands exactly on 1 - 2^-8.
     const float kFixFactor = 0.99609375f;
-
-    float m = kNegInf;    // running max of the raw scores S
-    int cnt = 0;          // how many seen scores equal m
-    float ms = kNegInf;   // m * scale_log2: the shift without the fix
-    bool raised = false;  // the shift in use is ms + delta (fix active on this row)
-    float l = 0.f;        // running sum of the unrounded P, relative to the shift in use
-    bool ever_repeated = false;   // the running max occurred >= 2 times at some tile
+    uint32_t it_cnt = 0;   // softmax iterations done by this warpgroup
     bool ok = true;
 
-    for (int j = 0; j < n_t; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wd));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t r[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, r[c]);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_wait(r[c]);
-      float s[128];
-#pragma unroll
-      for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(r[i >> 5][i & 31]);
+    for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd)) {
+      const FwdItem w = fwd_item(p, item);
+      const int n_t = t ? w.n1 : w.n0;
+      if (n_t == 0) continue;
+      const int row = w.q0_row + t * 128 + (warp & 3) * 32 + lane;
+      const int limit = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
 
-      const int key0 = j * 128;
-      const bool masked = key0 + 127 > limit;
-      if (masked) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) s[i] = (key0 + i > limit) ? kNegInf : s[i];
-      }
-      // tile maximum: eight 16-wide 3-input max chains, then a short tree
-      float mx[8];
-#pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        float a = fmax3(s[16 * g], s[16 * g + 1], s[16 * g + 2]);
-#pragma unroll
-        for (int i = 3; i < 15; i += 2) a = fmax3(a, s[16 * g + i], s[16 * g + i + 1]);
-        mx[g] = fmaxf(a, s[16 * g + 15]);
-      }
-      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-      const float m_new = fmaxf(m, mt);
-      const float ms_new = (m_new == kNegInf) ? 0.f : m_new * sl2;
+      float m = kNegInf;    // running max of the raw scores S
+      int cnt = 0;          // how many seen scores equal m
+      float ms = kNegInf;   // m * scale_log2: the shift without the fix
+      bool raised = false;  // the shift in use is ms + delta (fix active on this row)
+      float l = 0.f;        // running sum of the unrounded P, relative to the shift in use
+      bool ever_repeated = false;   // the running max occurred >= 2 times at some tile
 
-      // P = 2^(S*scale_log2 - ms_new) in pairs; row sum and the count of
-      // entries equal to the tile max ride along as independent adds
-      const uint64_t c2 = f2_pack(sl2, sl2);
-      const uint64_t b2 = f2_pack(-ms_new, -ms_new);
-      uint64_t sum2[4] = {0, 0, 0, 0};
-      uint64_t eq2[2] = {0, 0};
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float x0 = fmaf(s[2 * i], sl2, -ms_new);
-        const float x1 = fmaf(s[2 * i + 1], sl2, -ms_new);
-        const float e0 = (s[2 * i] == mt) ? 1.f : 0.f;
-        const float e1 = (s[2 * i + 1] == mt) ? 1.f : 0.f;
-        eq2[i & 1] = f2_add(eq2[i & 1], f2_pack(e0, e1));
-        s[2 * i] = ex2(x0);
-        s[2 * i + 1] = ex2(x1);
-        sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(s[2 * i], s[2 * i + 1]));
-      }
-      float ea, eb, ec, ed;
-      f2_unpack(f2_add(eq2[0], eq2[1]), ea, eb);
-      const int ct = (mt == kNegInf) ? 0 : int(ea + eb);
-      int c_new = (m == m_new ? cnt : 0) + (mt == m_new ? ct : 0);
-      if (m_new == kNegInf) c_new = 0;
-      ever_repeated |= (c_new >= 2);
-      const bool raise = p.fix && c_new >= 2;
-      f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), ea, eb);
-      float rs = ea + eb;
-      if (__any_sync(0xffffffffu, raise)) {
-        // Rare path: some row of this warp has a repeated maximum.  S is still
-        // intact in TMEM; recompute P for the whole warp (unchanged rows get
-        // the identical arithmetic) and scale the repeated rows by 2^-delta.
-        uint32_t q[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, q[c]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_wait(q[c]);
-        float rs_raised = 0.f;
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const float sv = (masked && key0 + i > limit) ? kNegInf : __uint_as_float(q[i >> 5][i & 31]);
-          const float pv = ex2(fmaf(sv, sl2, -ms_new));
-          s[i] = raise ? pv * kFixFactor : pv;
-          rs_raised += s[i];
-        }
-        if (raise) rs = rs_raised;
-      }
-      // rescale of the running O and l: exact, whenever the shift moves
-      float alpha = ex2(ms - ms_new);
-      if (raise != raised) alpha = raise ? alpha * kFixFactor : alpha / kFixFactor;
-      (void)ec;
-      (void)ed;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]);
-        tmem_st16(t_s + c * 16, pk);
-      }
-      l = l * alpha + rs;
-      tmem_st_wait();
-
-      if (j > 0) {
-        // O_t must hold the finished P_bar V of tile j-1 before it is rescaled
-        ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (j - 1) & 1, wd));
+      for (int j = 0; j < n_t; ++j) {
+        const uint32_t ph = (it_cnt + j) & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], ph, wd));
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          const uint64_t a2 = f2_pack(alpha, alpha);
+        uint32_t r[4][32];
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_o + c * 32, o);
-            tmem_ld_wait(o);
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, r[c]);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float y0, y1;
-              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), y0, y1);
-              o[2 * i] = __float_as_uint(y0);
-              o[2 * i + 1] = __float_as_uint(y1);
-            }
-            tmem_st32(t_o + c * 32, o);
-          }
-          tmem_st_wait();
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
-      m = m_new;
-      cnt = c_new;
-      ms = ms_new;
-      raised = raise;
-    }
+        for (int c = 0; c < 4; ++c) tmem_ld_wait(r[c]);
+        float s[128];
+#pragma unroll
+        for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(r[i >> 5][i & 31]);
 
-    if (ok && n_t > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (n_t - 1) & 1, wd));
-      if (ok) {
-        tc_fence_after();
-        const float inv_l = 1.f / l;
-        __nv_bfloat16* orow = p.o + (size_t(bh) * p.N + row) * D;
+        const int key0 = j * 128;
+        const bool masked = key0 + 127 > limit;
+        if (masked) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(t_o + c * 32, o);
-          tmem_ld_wait(o);
-          uint32_t w[16];
+          for (int i = 0; i < 128; ++i) s[i] = (key0 + i > limit) ? kNegInf : s[i];
+        }
+        // tile maximum: eight 16-wide 3-input max chains, then a short tree
+        float mx[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            w[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-          if (row < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        for (int g = 0; g < 8; ++g) {
+          float a = fmax3(s[16 * g], s[16 * g + 1], s[16 * g + 2]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          for (int i = 3; i < 15; i += 2) a = fmax3(a, s[16 * g + i], s[16 * g + i + 1]);
+          mx[g] = fmaxf(a, s[16 * g + 15]);
+        }
+        const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+        const float m_new = fmaxf(m, mt);
+        const float ms_new = (m_new == kNegInf) ? 0.f : m_new * sl2;
+
+        // P = 2^(S*scale_log2 - ms_new); the row sum and the count of entries
+        // equal to the tile max ride along as independent packed adds
+        uint64_t sum2[4] = {0, 0, 0, 0};
+        uint64_t eq2[2] = {0, 0};
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float x0 = fmaf(s[2 * i], sl2, -ms_new);
+          const float x1 = fmaf(s[2 * i + 1], sl2, -ms_new);
+          const float e0 = (s[2 * i] == mt) ? 1.f : 0.f;
+          const float e1 = (s[2 * i + 1] == mt) ? 1.f : 0.f;
+          eq2[i & 1] = f2_add(eq2[i & 1], f2_pack(e0, e1));
+          s[2 * i] = ex2(x0);
+          s[2 * i + 1] = ex2(x1);
+          sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(s[2 * i], s[2 * i + 1]));
+        }
+        float ea, eb;
+        f2_unpack(f2_add(eq2[0], eq2[1]), ea, eb);
+        const int ct = (mt == kNegInf) ? 0 : int(ea + eb);
+        int c_new = (m == m_new ? cnt : 0) + (mt == m_new ? ct : 0);
+        if (m_new == kNegInf) c_new = 0;
+        ever_repeated |= (c_new >= 2);
+        const bool raise = p.fix && c_new >= 2;
+        f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), ea, eb);
+        float rs = ea + eb;
+        if (__any_sync(0xffffffffu, raise)) {
+          // Rare path: some row of this warp has a repeated maximum.  S is still
+          // intact in TMEM; recompute P for the whole warp (unchanged rows get
+          // the identical arithmetic) and scale the repeated rows by 2^-delta.
+          uint32_t q[4][32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, q[c]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld_wait(q[c]);
+          float rs_raised = 0.f;
+#pragma unroll
+          for (int i = 0; i < 128; ++i) {
+            const float sv = (masked && key0 + i > limit) ? kNegInf : __uint_as_float(q[i >> 5][i & 31]);
+            const float pv = ex2(fmaf(sv, sl2, -ms_new));
+            s[i] = raise ? pv * kFixFactor : pv;
+            rs_raised += s[i];
+          }
+          if (raise) rs = rs_raised;
+        }
+        // rescale of the running O and l: exact, whenever the shift moves
+        float alpha = ex2(ms - ms_new);
+        if (raise != raised) alpha = raise ? alpha * kFixFactor : alpha / kFixFactor;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]);
+          tmem_st16(t_s + c * 16, pk);
+        }
+        l = l * alpha + rs;
+        tmem_st_wait();
+
+        if (j > 0) {
+          // O_t must hold the finished P_bar V of tile j-1 before it is rescaled
+          ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (it_cnt + j - 1) & 1, wd));
+          if (!ok) break;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(t_o + c * 32, o);
+              tmem_ld_wait(o);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                float y0, y1;
+                f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), y0, y1);
+                o[2 * i] = __float_as_uint(y0);
+                o[2 * i + 1] = __float_as_uint(y1);
+              }
+              tmem_st32(t_o + c * 32, o);
+            }
+            tmem_st_wait();
           }
         }
-        if (row < p.N) {
-          p.lse[size_t(bh) * p.N + row] = (ms + (raised ? p.delta_log2 : 0.f) + lg2(l)) * kLn2;
-          if (p.ties) p.ties[size_t(bh) * p.N + row] = cnt | (ever_repeated ? (1 << 30) : 0);
-        }
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+        m = m_new;
+        cnt = c_new;
+        ms = ms_new;
+        raised = raise;
       }
+      if (!ok) break;
+
+      // epilogue: O = O_acc / l -> bf16; LSE in natural-log units
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (it_cnt + n_t - 1) & 1, wd));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t ow[D / 2];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_o + c * 32, o);
+        tmem_ld_wait(o);
+        const float inv_l = 1.f / l;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          ow[c * 16 + i] = pack_bf16(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+      }
+      // O_t is in registers: the next item's first P_bar V may overwrite it
+      tc_fence_before();
+      mbar_arrive(&o_free[t]);
+      if (row < p.N) {
+        uint4* dst = reinterpret_cast<uint4*>(p.o + (size_t(w.bh) * p.N + row) * D);
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(ow[4 * i], ow[4 * i + 1], ow[4 * i + 2], ow[4 * i + 3]);
+        p.lse[size_t(w.bh) * p.N + row] = (ms + (raised ? p.delta_log2 : 0.f) + lg2(l)) * kLn2;
+        if (p.ties) p.ties[size_t(w.bh) * p.N + row] = cnt | (ever_repeated ? (1 << 30) : 0);
+      }
+      it_cnt += n_t;
     }
   }
 

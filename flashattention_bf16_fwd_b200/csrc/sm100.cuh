@@ -348,6 +348,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
+// Work item that a persistent CTA takes in round `rnd` when items are sorted
+// heavy first: the CTAs sweep the sorted list back and forth (0..G-1, then
+// G-1..0, ...), so every CTA receives a mix of heavy and light items.
+__device__ __forceinline__ int snake_item(int rnd) {
+  const int g = int(gridDim.x);
+  const int c = int(blockIdx.x);
+  return rnd * g + ((rnd & 1) ? g - 1 - c : c);
+}
+
 // Per-warpgroup register reallocation (all four warps of a warpgroup execute
 // it).  An increase waits until decreases elsewhere in the CTA have returned
 // enough registers to the pool the CTA was launched with.
