@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(512, 1)
 
   if (warp >= 12) {
     // Producer and MMA warps need few registers; give them back first.
-    regs_decrease<L::kOtherRegs>();
+    regs_set<L::kOtherRegs, L::kLaunchRegs>();
     if (warp == 12) {
       // ----------------------------------------------------------- producer
       const uint64_t pol_kv = l2_policy_evict_first();
@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(512, 1)
       __syncwarp();
     }
   } else if (warp < 8) {
-    regs_increase<L::kComputeRegs>();
+    regs_set<L::kComputeRegs, L::kLaunchRegs>();
     // ------------------------------------------------------- key-row math
     const int quarter = warp & 3;
     const int half = warp >> 2;                      // queries 64*half .. +63
@@ -502,7 +502,7 @@ __global__ void __launch_bounds__(512, 1)
       }
     }
   } else {
-    regs_decrease<L::kDrainRegs>();
+    regs_set<L::kDrainRegs, L::kLaunchRegs>();
     // ------------------------------------------- dQ drain and dK/dV epilogue
     const int wq = warp & 3;
     const int rr = wq * 32 + lane;                   // query row (dQ) / key row (dK, dV)

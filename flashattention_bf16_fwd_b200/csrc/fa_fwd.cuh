@@ -53,6 +53,14 @@ struct FwdLayout {
   static constexpr int kBytes = kBarOff + 256;
   static constexpr int kAlloc = kBytes + 1024;        // room to align the base to 1 KB
   static constexpr uint32_t kTmemCols = 512;
+  // TMEM columns.  d = 64: S0, S1, P_bar0, P_bar1, O0, O1 each have their own,
+  // so S of the next key tile can be computed as soon as the softmax has read
+  // S of this one.  d = 128: O0, O1 take 256 columns and P_bar overwrites the
+  // first half of S; the next S then waits for P_bar V.
+  static constexpr bool kSepP = (D == 64);
+  __host__ __device__ static constexpr uint32_t tm_s(int t) { return 128 * t; }
+  __host__ __device__ static constexpr uint32_t tm_p(int t) { return kSepP ? 256 + 64 * t : 128 * t; }
+  __host__ __device__ static constexpr uint32_t tm_o(int t) { return kSepP ? 384 + 64 * t : 256 + D * t; }
   static constexpr int kThreads = 384;
   static constexpr int kLaunchRegs = 168;       // per thread, fixed by __launch_bounds__(384, 1)
   static constexpr uint32_t kSoftmaxRegs = 208;
@@ -98,7 +106,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* p_full = s_full + 2;             // [2]
   uint64_t* o_done = p_full + 2;             // [2]
   uint64_t* o_free = o_done + 2;             // [2]
-  uint64_t* mma_done = o_free + 2;
+  uint64_t* s_free = o_free + 2;             // [2] the softmax has read S_t (d = 64)
+  uint64_t* mma_done = s_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -118,6 +127,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&p_full[t], 128);
       mbar_init(&o_done[t], 1);
       mbar_init(&o_free[t], 128);
+      mbar_init(&s_free[t], 128);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -140,7 +150,7 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp >= 8) {
     // Producer and MMA warps need few registers; give them back first.
-    regs_decrease<L::kOtherRegs>();
+    regs_set<L::kOtherRegs, L::kLaunchRegs>();
     if (warp == 8) {
       // ------------------------------------------------------------- producer
       if (lane == 0) {
@@ -177,25 +187,26 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) {
         constexpr uint32_t kIdS = make_idesc_bf16(128, 128, 0, 0);   // Q K^T: both K-major
         constexpr uint32_t kIdPV = make_idesc_bf16(128, D, 0, 1);    // P_bar V: V is MN-major
-        const uint32_t sq = smem_u32(smem + L::kQOff);
-        const uint32_t skv = smem_u32(smem + L::kKVOff);
+        // Descriptors are built once; each MMA only advances the start address.
+        const uint64_t dq0 = make_sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
+        const uint64_t dk0 = make_sdesc_sw128(smem_u32(smem + L::kKVOff), 16, 1024);
+        const uint64_t dv0 = make_sdesc_sw128(smem_u32(smem + L::kKVOff + L::kTileBytes), L::kSubBytes, 1024);
         auto issue_s = [&](int t, uint32_t st) {
-          const uint32_t qa = sq + t * L::kTileBytes;
-          const uint32_t ka = skv + st * 2 * L::kTileBytes;
+          const uint64_t a = sdesc_add(dq0, t * L::kTileBytes);
+          const uint64_t b = sdesc_add(dk0, st * 2 * L::kTileBytes);
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t off = (k >> 2) * L::kSubBytes + (k & 3) * 32;
-            umma_ss(tmem + t * 128, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
-                    kIdS, k > 0);
+            umma_ss(tmem + L::tm_s(t), sdesc_add(a, off), sdesc_add(b, off), kIdS, k > 0);
           }
           umma_commit(&s_full[t]);
         };
         auto issue_pv = [&](int t, uint32_t st, int j) {
-          const uint32_t va = skv + st * 2 * L::kTileBytes + L::kTileBytes;
+          const uint64_t b = sdesc_add(dv0, st * 2 * L::kTileBytes);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts(tmem + 256 + t * D, tmem + t * 128 + k * 8,
-                    make_sdesc_sw128(va + k * 2048, L::kSubBytes, 1024), kIdPV, (j > 0 || k > 0) ? 1u : 0u);
+            umma_ts(tmem + L::tm_o(t), tmem + L::tm_p(t) + k * 8, sdesc_add(b, k * 2048), kIdPV,
+                    (j > 0 || k > 0) ? 1u : 0u);
           umma_commit(&o_done[t]);
         };
         uint32_t kv_cnt = 0;           // K/V tiles consumed
@@ -210,14 +221,33 @@ __global__ void __launch_bounds__(384, 1)
                      mbar_wait(&kv_full[kv_cnt % L::kStages], (kv_cnt / L::kStages) & 1, wd)))
             break;
           tc_fence_after();
-          for (int t = 0; t < 2; ++t)
-            if (nt[t] > 0) issue_s(t, kv_cnt % L::kStages);
-          if (w.nmax == 1) umma_commit(q_empty);
+          for (int t = 0; t < 2; ++t) {
+            if (nt[t] == 0) continue;
+            // d=64: the softmax must have read the last S_t of the previous item
+            if (L::kSepP && it_cnt[t] > 0 && !(ok = mbar_wait(&s_free[t], (it_cnt[t] - 1) & 1, wd))) break;
+            issue_s(t, kv_cnt % L::kStages);
+          }
+          if (ok && w.nmax == 1) umma_commit(q_empty);
           for (int j = 0; ok && j < w.nmax; ++j) {
             const uint32_t st = (kv_cnt + j) % L::kStages;
             const uint32_t stn = (kv_cnt + j + 1) % L::kStages;
-            for (int t = 0; t < 2; ++t) {
-              if (j < nt[t]) {
+            if (L::kSepP) {
+              // S of key tile j+1 as soon as the softmax has read S of tile j;
+              // then P_bar V of tile j
+              if (j + 1 < w.nmax) {
+                const uint32_t nxt = kv_cnt + j + 1;
+                if (!(ok = mbar_wait(&kv_full[stn], (nxt / L::kStages) & 1, wd))) break;
+                for (int t = 0; t < 2; ++t) {
+                  if (j + 1 >= nt[t]) continue;
+                  if (!(ok = mbar_wait(&s_free[t], (it_cnt[t] + j) & 1, wd))) break;
+                  tc_fence_after();
+                  issue_s(t, stn);
+                }
+                if (!ok) break;
+                if (j + 2 == w.nmax) umma_commit(q_empty);   // the item's last S MMAs are issued
+              }
+              for (int t = 0; t < 2; ++t) {
+                if (j >= nt[t]) continue;
                 if (!(ok = mbar_wait(&p_full[t], (it_cnt[t] + j) & 1, wd))) break;
                 // the first P_bar V of an item overwrites O_t: the previous
                 // item's epilogue must have read it
@@ -225,16 +255,27 @@ __global__ void __launch_bounds__(384, 1)
                 tc_fence_after();
                 issue_pv(t, st, j);
               }
-              if (t == 0 && j + 1 < w.nmax) {
-                const uint32_t nxt = kv_cnt + j + 1;
-                if (!(ok = mbar_wait(&kv_full[stn], (nxt / L::kStages) & 1, wd))) break;
-                tc_fence_after();
-                if (j + 1 < nt[0]) issue_s(0, stn);
-              }
-              if (t == 1) {
-                umma_commit(&kv_empty[st]);
-                if (j + 1 < nt[1]) issue_s(1, stn);
-                if (j + 2 == w.nmax) umma_commit(q_empty);   // the item's last S MMAs are issued
+              if (!ok) break;
+              umma_commit(&kv_empty[st]);
+            } else {
+              for (int t = 0; t < 2; ++t) {
+                if (j < nt[t]) {
+                  if (!(ok = mbar_wait(&p_full[t], (it_cnt[t] + j) & 1, wd))) break;
+                  if (j == 0 && !(ok = mbar_wait(&o_free[t], (ep_cnt[t] & 1) ^ 1, wd))) break;
+                  tc_fence_after();
+                  issue_pv(t, st, j);
+                }
+                if (t == 0 && j + 1 < w.nmax) {
+                  const uint32_t nxt = kv_cnt + j + 1;
+                  if (!(ok = mbar_wait(&kv_full[stn], (nxt / L::kStages) & 1, wd))) break;
+                  tc_fence_after();
+                  if (j + 1 < nt[0]) issue_s(0, stn);   // S_0 of tile j+1 overwrites P_bar_0 after P_bar V
+                }
+                if (t == 1) {
+                  umma_commit(&kv_empty[st]);
+                  if (j + 1 < nt[1]) issue_s(1, stn);
+                  if (j + 2 == w.nmax) umma_commit(q_empty);   // the item's last S MMAs are issued
+                }
               }
             }
           }
@@ -251,12 +292,13 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     }
   } else {
-    regs_increase<L::kSoftmaxRegs>();
+    regs_set<L::kSoftmaxRegs, L::kLaunchRegs>();
     // --------------------------------------------------- softmax warpgroups
     const int t = warp >> 2;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
-    const uint32_t t_s = tmem + lane_base + uint32_t(t * 128);
-    const uint32_t t_o = tmem + lane_base + uint32_t(256 + t * D);
+    const uint32_t t_s = tmem + lane_base + L::tm_s(t);
+    const uint32_t t_p = tmem + lane_base + L::tm_p(t);
+    const uint32_t t_o = tmem + lane_base + L::tm_o(t);
     const float sl2 = p.scale_log2;
     // 2^-delta: on a repeated-max row P is computed with the plain shift and
     // then multiplied by this, which is the same as raising m by delta; each
@@ -355,43 +397,46 @@ __global__ void __launch_bounds__(384, 1)
           }
           if (raise) rs = rs_raised;
         }
+        if (L::kSepP) {                                // S_t is read: the next S may overwrite it
+          tc_fence_before();
+          mbar_arrive(&s_free[t]);
+        }
         // rescale of the running O and l: exact, whenever the shift moves
         float alpha = ex2(ms - ms_new);
         if (raise != raised) alpha = raise ? alpha * kFixFactor : alpha / kFixFactor;
+        l = l * alpha + rs;
+        if (j > 0) {
+          // P_bar V of tile j-1 must be finished: it read the P_bar buffer and
+          // O_t must hold its result before O_t is rescaled
+          ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (it_cnt + j - 1) & 1, wd));
+          if (!ok) break;
+          tc_fence_after();
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]);
-          tmem_st16(t_s + c * 16, pk);
+          tmem_st16(t_p + c * 16, pk);
         }
-        l = l * alpha + rs;
-        tmem_st_wait();
-
-        if (j > 0) {
-          // O_t must hold the finished P_bar V of tile j-1 before it is rescaled
-          ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (it_cnt + j - 1) & 1, wd));
-          if (!ok) break;
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
-            const uint64_t a2 = f2_pack(alpha, alpha);
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c * 32, o);
+            tmem_ld_wait(o);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(t_o + c * 32, o);
-              tmem_ld_wait(o);
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                float y0, y1;
-                f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), y0, y1);
-                o[2 * i] = __float_as_uint(y0);
-                o[2 * i + 1] = __float_as_uint(y1);
-              }
-              tmem_st32(t_o + c * 32, o);
+            for (int i = 0; i < 16; ++i) {
+              float y0, y1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), y0, y1);
+              o[2 * i] = __float_as_uint(y0);
+              o[2 * i + 1] = __float_as_uint(y1);
             }
-            tmem_st_wait();
+            tmem_st32(t_o + c * 32, o);
           }
         }
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&p_full[t]);
         m = m_new;

@@ -79,16 +79,17 @@ struct Watchdog {
 // Wait until the phase with parity `parity` of `bar` has completed.  Returns
 // false (and marks the CTA aborted, and records kDevErrTimeout) when the wait
 // exceeds kWaitTimeoutNs, or when another role of the CTA already aborted.
+// The clock is read only every 1024 polls, so that each wait site stays small.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Watchdog& wd) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
   uint32_t spins = 0;
+  uint64_t deadline = 0;
   while (!mbar_try_wait(bar, parity)) {
-    if ((++spins & 15u) == 0) {
-      if (*wd.abort) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+    if ((++spins & 1023u) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (deadline == 0) deadline = now + kWaitTimeoutNs;
+      if (*wd.abort || now > deadline) {
+        if (!*wd.abort) atomicExch(wd.dev_error, kDevErrTimeout);
         *wd.abort = 1;
-        atomicExch(wd.dev_error, kDevErrTimeout);
         return false;
       }
     }
@@ -234,6 +235,11 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
   return d;
 }
 
+// A descriptor advanced by `bytes` along its start address (bits 0-13 hold
+// address >> 4; shared-memory addresses stay below 256 KB, so no carry
+// leaves the field).
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
 #define FA_R8(i) "=r"(r[i + 0]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), \
                  "=r"(r[i + 6]), "=r"(r[i + 7])
 #define FA_W8(i) "+r"(r[i + 0]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]), \
@@ -357,17 +363,22 @@ __device__ __forceinline__ int snake_item(int rnd) {
   return rnd * g + ((rnd & 1) ? g - 1 - c : c);
 }
 
-// Per-warpgroup register reallocation (all four warps of a warpgroup execute
-// it).  An increase waits until decreases elsewhere in the CTA have returned
-// enough registers to the pool the CTA was launched with.
-template <uint32_t kRegs>
-__device__ __forceinline__ void regs_increase() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-
-template <uint32_t kRegs>
-__device__ __forceinline__ void regs_decrease() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+// Per-warpgroup register reallocation from the launch count kLaunch to kNew
+// (all four warps of a warpgroup execute it).  The direction is chosen at
+// compile time: setmaxnreg.dec must never ask for more than the current
+// count, setmaxnreg.inc never for less.  An increase waits until decreases
+// elsewhere in the CTA have returned enough registers to the pool the CTA
+// was launched with.
+template <uint32_t kNew, uint32_t kLaunch>
+__device__ __forceinline__ void regs_set() {
+  static_assert(kNew % 8 == 0 && kNew >= 24 && kNew <= 256, "setmaxnreg count out of range");
+  if constexpr (kNew == kLaunch) {
+    // nothing to move
+  } else if constexpr (kNew > kLaunch) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kNew));
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kNew));
+  }
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
