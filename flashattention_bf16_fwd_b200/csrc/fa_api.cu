@@ -298,6 +298,8 @@ const char* fa_status_string(int status) {
     case FA_ERR_TIMEOUT: return "a kernel gave up on a bounded wait (device error flag set)";
     case FA_ERR_ARG: return "causal must be 0 or 1 and scale finite and > 0";
     case FA_ERR_DEVICE: return "no sm_100 device, or tensor-map encoding unavailable";
+    case FA_ERR_SCRATCH_LIMIT:
+      return "fa_bwd_noalloc: fa_bwd_workspace_size() exceeds FA_BWD_NOALLOC_SCRATCH_BYTES (32 MiB)";
     default: return "unknown status";
   }
 }
@@ -317,3 +319,60 @@ int fa_check_device_error(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// fa_bwd_noalloc: the backward pass for callers that cannot allocate device
+// memory (an allocator owned by a host application, a fixed memory budget
+// reserved at start-up, a real-time loop that must not enter the driver's
+// allocator).  Its scratch is a fixed device global instead of a workspace
+// argument.
+
+namespace fa {
+namespace {
+
+// The FP32 dQ accumulator and D for fa_bwd_noalloc.  Every GPU that loads
+// this library holds it until the process exits.  In host code this name is
+// only a handle for cudaGetSymbolAddress, never a device address.
+__device__ __align__(256) uint8_t g_bwd_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
+
+struct ScratchState {
+  std::once_flag once;
+  void* ptr = nullptr;   // device address of g_bwd_scratch on this device
+};
+ScratchState g_scratch[kMaxDevices];
+
+// Looked up once per device, on the first fa_bwd_noalloc call made with that
+// device current.  The lookup may load the module, so that first call must
+// not happen inside a stream capture.
+void* bwd_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  ScratchState* st = &g_scratch[dev];
+  std::call_once(st->once, [st] {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) == cudaSuccess) st->ptr = ptr;
+  });
+  return st->ptr;
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                              const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                              int causal, float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
+  const int rc = check_common(B, H, N, d, causal, scale);
+  if (rc != FA_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_ALIGN;
+  if (fa_bwd_workspace_size(B, H, N, d) > FA_BWD_NOALLOC_SCRATCH_BYTES) return FA_ERR_SCRATCH_LIMIT;
+  if (!device_state()) return FA_ERR_DEVICE;
+  void* scratch = bwd_scratch();
+  if (!scratch) return FA_ERR_DEVICE;
+  // fa_bwd's first launch zeroes the accumulator and rewrites D, so what the
+  // previous call left in the array does not matter.
+  return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, scratch, FA_BWD_NOALLOC_SCRATCH_BYTES, B, H, N, d, causal,
+                scale, stream);
+}

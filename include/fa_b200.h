@@ -63,8 +63,10 @@ typedef enum {
   FA_ERR_LAUNCH = -7,    /* the CUDA runtime refused a launch                 */
   FA_ERR_TIMEOUT = -8,   /* a kernel's bounded wait expired (device flag)     */
   FA_ERR_ARG = -9,       /* causal not in {0,1}, or scale not finite and > 0  */
-  FA_ERR_DEVICE = -10    /* no sm_100 device, or the driver entry point for
+  FA_ERR_DEVICE = -10,   /* no sm_100 device, or the driver entry point for
                             tensor maps is unavailable                        */
+  FA_ERR_SCRATCH_LIMIT = -11 /* fa_bwd_noalloc: the problem needs more scratch
+                            than FA_BWD_NOALLOC_SCRATCH_BYTES                 */
 } fa_status;
 
 /*
@@ -136,6 +138,41 @@ FA_API int fa_bwd_main(const void* q, const void* k, const void* v,
                        int N, int d, int causal, float scale, void* stream);
 FA_API int fa_bwd_finish(void* dq, const void* workspace, size_t workspace_bytes,
                          int B, int H, int N, int d, float scale, void* stream);
+
+/*
+ * fa_bwd_noalloc - fa_bwd for callers that must not allocate device memory.
+ * The paper has no counterpart: this is an interface convenience.
+ *
+ * Who needs it: code that runs where cudaMalloc is off limits - a plugin
+ * inside a host that owns all device memory through its own pool, a process
+ * whose allocator is reserved up front to a fixed budget, or a real-time loop
+ * that must not take the driver's allocation locks.  fa_bwd asks such a
+ * caller for a workspace it has no way to get; this call needs none.
+ *
+ * Arguments and results are those of fa_bwd without workspace/workspace_bytes.
+ * The scratch (FP32 dQ accumulator and D) lives instead in one fixed array of
+ * FA_BWD_NOALLOC_SCRATCH_BYTES (32 MiB) compiled into the library as a
+ * device global: every GPU that loads the library holds those 32 MiB until
+ * the process exits, whether or not this call is used.
+ *   - Limit: fa_bwd_workspace_size(B,H,N,d) <= FA_BWD_NOALLOC_SCRATCH_BYTES,
+ *     which allows B*H*N <= 129055 rows at d = 64 (8 x 12 x 1024 = 98304
+ *     fits) and <= 65027 rows at d = 128.  Larger problems return
+ *     FA_ERR_SCRATCH_LIMIT and launch nothing.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on a device (the current device) looks up the array's
+ *     device address once; make that first call before any stream capture
+ *     begins on that device.
+ *   - The array is shared by every call on a device and keeps the last call's
+ *     contents; each call clears the accumulator before use.  Calls whose
+ *     kernels overlap on the GPU (concurrent streams, or host threads without
+ *     stream ordering between them) race on the array and give wrong
+ *     gradients: order them on one stream, or serialise them.
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+FA_API int fa_bwd_noalloc(const void* q, const void* k, const void* v,
+                          const void* o, const float* lse, const void* dout,
+                          void* dq, void* dk, void* dv, int B, int H, int N,
+                          int d, int causal, float scale, void* stream);
 
 /* fa_status_string - static, NUL-terminated description of a status code. */
 FA_API const char* fa_status_string(int status);

@@ -33,7 +33,7 @@ def declared_symbols():
 def test_header_declares_the_boundary():
     assert declared_symbols() == sorted(["fa_fwd", "fa_fwd_ties", "fa_bwd_workspace_size", "fa_bwd",
                                          "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish",
-                                         "fa_status_string", "fa_check_device_error"])
+                                         "fa_bwd_noalloc", "fa_status_string", "fa_check_device_error"])
 
 
 def test_library_exports_every_declared_symbol(fa):
@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(fa):
 
 
 def test_status_strings(fa):
-    for code in range(0, -11, -1):
+    for code in range(0, -12, -1):
         s = fa.fa_status_string(code)
         assert s and s != "unknown status"
     assert fa.fa_status_string(-99) == "unknown status"
@@ -106,11 +106,30 @@ def test_bwd_argument_errors(fa):
     assert fa.lib.fa_bwd_finish(A, A, ws, 1, 1, 128, 64, -1.0, None) == FA_ERR_ARG
 
 
+FA_ERR_SCRATCH_LIMIT = -11
+
+
+def test_bwd_noalloc_argument_errors(fa):
+    def nb(dq=A, N=128, d=64, H=1):
+        return fa.lib.fa_bwd_noalloc(A, A, A, A, A, A, dq, A, A, 1, H, N, d, 1, 0.125, None)
+
+    assert nb(dq=None) == FA_ERR_NULL
+    assert nb(d=96) == FA_ERR_HEADDIM
+    assert nb(dq=MIS) == FA_ERR_ALIGN
+    # the fixed 32 MiB scratch holds 129055 rows at d = 64 and 65027 at d = 128
+    assert nb(N=129056, d=64) == FA_ERR_SCRATCH_LIMIT
+    assert nb(N=65028, d=128) == FA_ERR_SCRATCH_LIMIT
+    assert nb(N=4096, H=32, d=128) == FA_ERR_SCRATCH_LIMIT
+    assert fa.fa_bwd_workspace_size(1, 1, 129055, 64) <= 32 << 20 < fa.fa_bwd_workspace_size(1, 1, 129056, 64)
+    assert fa.fa_bwd_workspace_size(1, 1, 65027, 128) <= 32 << 20 < fa.fa_bwd_workspace_size(1, 1, 65028, 128)
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
 def test_valid_call_without_gpu_reports_device_error(fa):
     assert fwd(fa) == FA_ERR_DEVICE
     ws = fa.fa_bwd_workspace_size(1, 1, 128, 64)
     assert fa.lib.fa_bwd(A, A, A, A, A, A, A, A, A, A, ws, 1, 1, 128, 64, 1, 0.125, None) == FA_ERR_DEVICE
+    assert fa.lib.fa_bwd_noalloc(A, A, A, A, A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, None) == FA_ERR_DEVICE
 
 
 def test_binding_rejects_cpu_tensors(fa):
