@@ -146,8 +146,10 @@ def test_deterministic_forward(fa):
     b = run_gpu(fa, x, bwd=True)
     for n in ("o", "lse", "dk", "dv"):
         assert np.array_equal(a[n], b[n]), n
-    # dQ is summed with atomics in an arbitrary order: equal up to rounding
-    assert normwise_rel_err(a["dq"], b["dq"]) < 1e-5
+    # dQ is summed with reduce-adds in an arbitrary order: the FP32 sums agree
+    # to rounding, and after the bf16 rounding of dQ an element differs by at
+    # most one bf16 step (2^-8 relative) unless its terms cancel
+    assert normwise_rel_err(a["dq"], b["dq"]) < 2.0 ** -8
 
 
 def test_outputs_stay_in_bounds(fa):

@@ -5,11 +5,12 @@ The file name sorts last so that it also runs after every other GPU test in
 one process; it passes on its own in a fresh process as well.  Two calls in a
 row on the same shape: the fixed scratch array keeps the first call's
 contents, so a second call that failed to clear its accumulator would show
-the first call's dQ in its own.  dK and dV do not depend on the scratch and
-must match fa_bwd bit for bit; dQ is summed with reduce-adds in an order that
-varies from run to run, so it is held to the same 1e-5 normwise bound as the
-run-to-run determinism test.  A d = 128 call follows to cover the other
-kernel instantiation.
+the first call's dQ in its own (an error of order 100%).  dK and dV do not
+depend on the scratch and must match fa_bwd bit for bit.  dQ is summed with
+reduce-adds in an order that varies from run to run, so after its rounding to
+bf16 a few elements land one bf16 step apart; it is held to the gradient
+tolerance of the parity tests (normwise 5e-2).  A d = 128 call follows to
+cover the other kernel instantiation.
 """
 import pytest
 import torch
@@ -19,7 +20,7 @@ from flashattention_bf16_fwd_b200.workloads import Workload, make_inputs
 
 pytestmark = pytest.mark.gpu
 
-RUN_TO_RUN_RTOL = 1e-5
+GRAD_RTOL = 5e-2
 
 
 def test_noalloc_matches_fa_bwd_on_calls_in_a_row():
@@ -43,4 +44,4 @@ def test_noalloc_matches_fa_bwd_on_calls_in_a_row():
         dq, dk, dv = got
         assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2]), (w, seed)
         err = normwise_rel_err(dq.float().cpu().numpy(), ref[0].float().cpu().numpy())
-        assert err <= RUN_TO_RUN_RTOL, (w, seed, err)
+        assert err <= GRAD_RTOL, (w, seed, err)
