@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "../../include/fa_b200.h"
 #include "fa_bwd.cuh"
@@ -85,6 +86,28 @@ DeviceState* device_state() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Every kernel is launched with programmatic stream serialisation: it may be
+// scheduled while the previous kernel in the stream drains, runs its set-up
+// (barriers, TMEM, descriptor prefetch), and waits in grid_dep_wait() before
+// it touches global memory.
+constexpr int kProgrammaticLaunch = 1;
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                   Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = kProgrammaticLaunch;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 int check_common(int B, int H, int N, int d, int causal, float scale) {
   if (d != 64 && d != 128) return FA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
@@ -153,11 +176,12 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   prm.fix = fix_mode;
   const int n_items = prm.n_pairs * BH;
   const dim3 grid(unsigned(n_items < st->num_sms ? n_items : st->num_sms));
-  if (d == 64)
-    fa_fwd_kernel<64><<<grid, FwdLayout<64>::kThreads, FwdLayout<64>::kAlloc, stream>>>(mq, mk, mv, prm);
-  else
-    fa_fwd_kernel<128><<<grid, FwdLayout<128>::kThreads, FwdLayout<128>::kAlloc, stream>>>(mq, mk, mv, prm);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+  const cudaError_t e =
+      (d == 64) ? launch(fa_fwd_kernel<64>, grid, dim3(FwdLayout<64>::kThreads), FwdLayout<64>::kAlloc, stream, mq, mk,
+                         mv, prm)
+                : launch(fa_fwd_kernel<128>, grid, dim3(FwdLayout<128>::kThreads), FwdLayout<128>::kAlloc, stream, mq,
+                         mk, mv, prm);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -202,10 +226,10 @@ int fa_bwd_preprocess(const void* o, const void* dout, void* workspace, size_t w
   float* dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256(rows * d * sizeof(float)));
   const int threads = 256;
   const long long blocks = ((long long)rows * 8 + threads - 1) / threads;
-  fa_bwd_pre_kernel<<<unsigned(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), dsum, dq_acc,
-      (long long)rows, d);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+  const cudaError_t e = launch(fa_bwd_pre_kernel, dim3(unsigned(blocks)), dim3(threads), 0,
+                               static_cast<cudaStream_t>(stream), static_cast<const __nv_bfloat16*>(o),
+                               static_cast<const __nv_bfloat16*>(dout), dsum, dq_acc, (long long)rows, d);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dout, void* dk,
@@ -242,11 +266,12 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, c
   const int n_items = prm.n_kv * BH;
   const dim3 grid(unsigned(n_items < st->num_sms ? n_items : st->num_sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 64)
-    fa_bwd_kernel<64><<<grid, BwdLayout<64>::kThreads, BwdLayout<64>::kAlloc, s>>>(mq, mk, mv, mdo, mdq, prm);
-  else
-    fa_bwd_kernel<128><<<grid, BwdLayout<128>::kThreads, BwdLayout<128>::kAlloc, s>>>(mq, mk, mv, mdo, mdq, prm);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+  const cudaError_t e =
+      (d == 64) ? launch(fa_bwd_kernel<64>, grid, dim3(BwdLayout<64>::kThreads), BwdLayout<64>::kAlloc, s, mq, mk, mv,
+                         mdo, mdq, prm)
+                : launch(fa_bwd_kernel<128>, grid, dim3(BwdLayout<128>::kThreads), BwdLayout<128>::kAlloc, s, mq, mk,
+                         mv, mdo, mdq, prm);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 int fa_bwd_finish(void* dq, const void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale,
@@ -260,9 +285,10 @@ int fa_bwd_finish(void* dq, const void* workspace, size_t workspace_bytes, int B
   if (!device_state()) return FA_ERR_DEVICE;
   const long long n8 = (long long)B * H * N * d / 8;
   const int threads = 256;
-  fa_bwd_dq_kernel<<<unsigned((n8 + threads - 1) / threads), threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const float*>(workspace), static_cast<__nv_bfloat16*>(dq), scale, n8);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+  const cudaError_t e = launch(fa_bwd_dq_kernel, dim3(unsigned((n8 + threads - 1) / threads)), dim3(threads), 0,
+                               static_cast<cudaStream_t>(stream), static_cast<const float*>(workspace),
+                               static_cast<__nv_bfloat16*>(dq), scale, n8);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,

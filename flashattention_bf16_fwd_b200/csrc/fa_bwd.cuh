@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
                                                          const __nv_bfloat16* __restrict__ dout,
                                                          float* __restrict__ dsum, float* __restrict__ dq_acc,
                                                          long long rows, int d) {
+  grid_dep_wait();
+  grid_dep_launch();
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long row = tid >> 3;
   const int sub = int(tid & 7);
@@ -60,6 +62,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
 __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict__ acc,
                                                         __nv_bfloat16* __restrict__ dq, float scale,
                                                         long long n8) {
+  grid_dep_wait();
+  grid_dep_launch();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n8) return;
   const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
@@ -232,6 +236,10 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // set-up above touched no global memory; from here on the previous
+  // kernel's writes are needed
+  grid_dep_wait();
+  grid_dep_launch();
   const Watchdog wd{abort_flag, p.dev_error};
 
   if (warp >= 12) {

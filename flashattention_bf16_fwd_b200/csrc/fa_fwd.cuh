@@ -146,6 +146,10 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // set-up above touched no global memory; from here on the previous
+  // kernel's writes are needed
+  grid_dep_wait();
+  grid_dep_launch();
   const Watchdog wd{abort_flag, p.dev_error};
 
   if (warp >= 8) {

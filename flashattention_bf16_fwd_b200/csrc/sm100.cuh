@@ -296,6 +296,20 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ----------------------------------------------------------------------------
+// programmatic dependent launch
+// ----------------------------------------------------------------------------
+// The library's kernels are launched so that each may be scheduled while the
+// kernel before it in the stream is still finishing.  grid_dep_wait() blocks
+// until that kernel (and so everything before it) has completed and its
+// writes are visible; a kernel must call it before it reads or writes global
+// memory.  Without the launch attribute it returns at once.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allows the next kernel in the stream to be scheduled now.  It still runs
+// grid_dep_wait() before touching memory, so this only hides launch latency.
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ----------------------------------------------------------------------------
 // arithmetic helpers
 // ----------------------------------------------------------------------------
 // 2^x with the MUFU unit (flush-to-zero; 2^-inf = +0).
