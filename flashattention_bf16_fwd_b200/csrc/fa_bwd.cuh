@@ -96,16 +96,20 @@ struct BwdLayout {
   // d=128 has no room and keeps one dO buffer, refilled after dV.
   static constexpr int kKVStages = (D == 64) ? 2 : 1;
   static constexpr int kDOStages = (D == 64) ? 2 : 1;
+  // Q_i (with its LSE and D rows) is loaded up to kQStages steps ahead;
+  // d=64 has room for a third stage, which hides the load behind a full step.
+  static constexpr int kQStages = (D == 64) ? 3 : 2;
   static constexpr int kKVOff = 0;                          // stage s: K, then V
-  static constexpr int kQOff = kKVStages * 2 * kTileBytes;  // 2 stages
-  static constexpr int kDOOff = kQOff + 2 * kTileBytes;
+  static constexpr int kQOff = kKVStages * 2 * kTileBytes;
+  static constexpr int kDOOff = kQOff + kQStages * kTileBytes;
   static constexpr int kDSOff = kDOOff + kDOStages * kTileBytes;   // dS, [128 keys][128 queries] bf16, MN-major
-  static constexpr int kStatOff = kDSOff + 2 * kSubBytes;  // 2 stages x (-LSE*log2e, D) x 128 floats
+  static constexpr int kStatOff = kDSOff + 2 * kSubBytes;  // kQStages x (-LSE*log2e, D) x 128 floats
   // dQ staging for the TMA reduce-add: per drain warp two 32 x 32 FP32 boxes
   static constexpr int kStageBox = 32 * 32 * 4;
-  static constexpr int kDQStageOff = kStatOff + 2 * 2 * 128 * 4;
+  static constexpr int kDQStageOff = kStatOff + kQStages * 2 * 128 * 4;
   static constexpr int kBarOff = kDQStageOff + 4 * 2 * kStageBox;
   static constexpr int kBytes = kBarOff + 256;
+  static_assert(kBytes <= 227 * 1024, "shared memory layout exceeds 227 KB");
   static constexpr int kAlloc = kBytes;                    // base is 1 KB aligned by declaration
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 512;
@@ -153,9 +157,11 @@ __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
 //               w%4) and queries 64*(w/4).. of each tile: P^T, dS^T
 //   warps 8-11  dQ drain (thread r owns query r; TMA reduce-add of 32 x 32
 //               FP32 boxes staged in shared memory) and the dK/dV epilogue
-//   warp  12    producer: K, V per item; Q_i, dO_i (TMA) plus LSE_i, D_i per step
+//   warp  12    producer: K, V per item; Q_i (TMA) plus LSE_i, D_i per step,
+//               up to kQStages steps ahead
+//   warp  14    producer: dO_i (TMA), independent of the Q ring
 //   warp  13    TMEM allocator + tcgen05.mma issuer
-//   warps 14-15 idle (complete the fourth warpgroup)
+//   warp  15    idle (completes the fourth warpgroup)
 // MMA order per query tile i (the tensor core runs the next tile's S while
 // the CUDA cores form dS_i, and dK_i, dQ_i, dP_{i+1} while they form P_{i+1}):
 //   dV_i += P_bar_i^T dO_i | S_{i+1} | dK_i += dS_i^T Q_i | dQ_i = dS_i K | dP_{i+1}
@@ -171,21 +177,21 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* kv_full = bars;        // [2]
   uint64_t* kv_empty = bars + 2;   // [2]
-  uint64_t* q_full = bars + 4;     // [2]
-  uint64_t* q_empty = bars + 6;    // [2]
-  uint64_t* do_full = bars + 8;    // [2]
-  uint64_t* do_empty = bars + 10;  // [2]
-  uint64_t* s_full = bars + 12;
-  uint64_t* p_full = bars + 13;
-  uint64_t* dp_full = bars + 14;
-  uint64_t* ds_full = bars + 15;
-  uint64_t* dq_full = bars + 16;
-  uint64_t* dq_free = bars + 17;
-  uint64_t* dkv_done = bars + 18;
-  uint64_t* dkv_free = bars + 19;
-  uint64_t* pt_free = bars + 20;
-  uint64_t* mma_done = bars + 21;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  uint64_t* do_full = bars + 4;    // [2]
+  uint64_t* do_empty = bars + 6;   // [2]
+  uint64_t* s_full = bars + 8;
+  uint64_t* p_full = bars + 9;
+  uint64_t* dp_full = bars + 10;
+  uint64_t* ds_full = bars + 11;
+  uint64_t* dq_full = bars + 12;
+  uint64_t* dq_free = bars + 13;
+  uint64_t* dkv_done = bars + 14;
+  uint64_t* dkv_free = bars + 15;
+  uint64_t* pt_free = bars + 16;
+  uint64_t* mma_done = bars + 17;
+  uint64_t* q_full = bars + 18;    // [kQStages]
+  uint64_t* q_empty = bars + 21;   // [kQStages]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* stats = reinterpret_cast<float*>(smem + L::kStatOff);   // [stage][-lse2 | dsum][128]
 
@@ -203,10 +209,12 @@ __global__ void __launch_bounds__(512, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
-      mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);
       mbar_init(&do_full[s], 1);
       mbar_init(&do_empty[s], 1);
+    }
+    for (int s = 0; s < L::kQStages; ++s) {
+      mbar_init(&q_full[s], 2);      // the Q tile's bytes, and the LSE/D rows in shared memory
+      mbar_init(&q_empty[s], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(p_full, 256);
@@ -267,10 +275,17 @@ __global__ void __launch_bounds__(512, 1)
           }
         }
         for (int it = 0; it < w.n_it; ++it, ++g) {
-          const uint32_t st = g & 1;
+          const uint32_t st = g % L::kQStages;
           const int q0 = (w.i_start + it) * 128;
-          ok = __all_sync(0xffffffffu, mbar_wait(&q_empty[st], ((g >> 1) & 1) ^ 1, wd));
+          ok = __all_sync(0xffffffffu, mbar_wait(&q_empty[st], ((g / L::kQStages) & 1) ^ 1, wd));
           if (!ok) break;
+          // the Q tile first, so that its load overlaps the LSE/D reads below
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&q_full[st], uint32_t(L::kTileBytes));
+            for (int s = 0; s < L::kSub; ++s)
+              tma_load_3d(smem + L::kQOff + st * L::kTileBytes + s * L::kSubBytes, &tm_q, &q_full[st], s * 64, q0,
+                          w.bh, pol_q);
+          }
           float* nlse = stats + st * 256;
           float* dd = nlse + 128;
 #pragma unroll
@@ -283,12 +298,18 @@ __global__ void __launch_bounds__(512, 1)
             dd[r] = in ? p.dsum[size_t(w.bh) * p.N + row] : 0.f;
           }
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&q_full[st], uint32_t(L::kTileBytes));
-            for (int s = 0; s < L::kSub; ++s)
-              tma_load_3d(smem + L::kQOff + st * L::kTileBytes + s * L::kSubBytes, &tm_q, &q_full[st], s * 64, q0,
-                          w.bh, pol_q);
-          }
+          if (lane == 0) mbar_arrive(&q_full[st]);   // second arrival: the rows are in shared memory
+        }
+      }
+    } else if (warp == 14) {
+      // ------------------------------------------------------- dO producer
+      const uint64_t pol_q = l2_policy_evict_last();
+      uint32_t g = 0;
+      bool ok = true;
+      for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd)) {
+        const BwdItem w = bwd_item(p, item);
+        for (int it = 0; it < w.n_it; ++it, ++g) {
+          const int q0 = (w.i_start + it) * 128;
           // dO_i: with a single buffer it is refilled once dV_{i-1} has read it
           const uint32_t sd = g % L::kDOStages;
           ok = __all_sync(0xffffffffu, mbar_wait(&do_empty[sd], ((g / L::kDOStages) & 1) ^ 1, wd));
@@ -308,19 +329,32 @@ __global__ void __launch_bounds__(512, 1)
         constexpr uint32_t kIdS = make_idesc_bf16(128, 128, 0, 0);   // K Q^T, V dO^T: K-major operands
         constexpr uint32_t kIdAcc = make_idesc_bf16(128, D, 0, 1);   // TMEM A x MN-major B (dV, dK)
         constexpr uint32_t kIdDQ = make_idesc_bf16(128, D, 1, 1);    // dS (MN-major) x K (MN-major)
-        const uint32_t sds = smem_u32(smem + L::kDSOff);
-        auto kmajor_mma = [&](uint32_t d_tm, uint32_t a, uint32_t b) {
+        // Descriptors as 32-bit low halves with one shared high half (every
+        // operand has a 1024-byte stride): this thread shares its issue slots
+        // with the busiest warps of the CTA, so each MMA costs it only an add.
+        // K-major operands use a leading byte offset of 16, MN-major ones the
+        // distance between 64-wide blocks.
+        constexpr uint32_t kHi = sdesc_hi(1024);
+        constexpr uint32_t kLboMN = uint32_t(L::kSubBytes >> 4) << 16;
+        constexpr uint32_t kLboK = uint32_t(16 >> 4) << 16;
+        const uint32_t ds_lo = sdesc_lo(smem_u32(smem + L::kDSOff), L::kSubBytes);
+        auto kmajor_mma = [&](uint32_t d_tm, uint32_t a_lo, uint32_t b_lo) {   // low halves without LBO
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k >> 2) * L::kSubBytes + (k & 3) * 32;
-            umma_ss(d_tm, make_sdesc_sw128(a + off, 16, 1024), make_sdesc_sw128(b + off, 16, 1024), kIdS, k > 0);
+            const uint32_t off = ((k >> 2) * L::kSubBytes + (k & 3) * 32) >> 4;
+            umma_ss_lh(d_tm, (a_lo + off) | kLboK, (b_lo + off) | kLboK, kHi, kIdS, k > 0 ? 1u : 0u);
           }
         };
-        auto q_of = [&](uint32_t gg) { return smem_u32(smem + L::kQOff + (gg & 1) * L::kTileBytes); };
-        auto do_of = [&](uint32_t gg) {
-          return smem_u32(smem + L::kDOOff + (gg % L::kDOStages) * L::kTileBytes);
+        // start-address halves (address >> 4) of each buffer
+        auto q_of = [&](uint32_t gg) {
+          return (smem_u32(smem + L::kQOff) >> 4) + (gg % L::kQStages) * (L::kTileBytes >> 4);
         };
-        auto wait_q = [&](uint32_t gg) { return mbar_wait(&q_full[gg & 1], (gg >> 1) & 1, wd); };
+        auto do_of = [&](uint32_t gg) {
+          return (smem_u32(smem + L::kDOOff) >> 4) + (gg % L::kDOStages) * (L::kTileBytes >> 4);
+        };
+        auto wait_q = [&](uint32_t gg) {
+          return mbar_wait(&q_full[gg % L::kQStages], (gg / L::kQStages) & 1, wd);
+        };
         auto wait_do = [&](uint32_t gg) {
           return mbar_wait(&do_full[gg % L::kDOStages], (gg / L::kDOStages) & 1, wd);
         };
@@ -330,8 +364,8 @@ __global__ void __launch_bounds__(512, 1)
         for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
           const BwdItem w = bwd_item(p, item);
           const uint32_t ks = n_done % L::kKVStages;
-          const uint32_t sk = smem_u32(smem + L::kKVOff + ks * 2 * L::kTileBytes);
-          const uint32_t sv = sk + L::kTileBytes;
+          const uint32_t sk = (smem_u32(smem + L::kKVOff) >> 4) + ks * (2 * L::kTileBytes >> 4);
+          const uint32_t sv = sk + (L::kTileBytes >> 4);
           if (!(ok = mbar_wait(&kv_full[ks], (n_done / L::kKVStages) & 1, wd) && wait_q(g) && wait_do(g))) break;
           tc_fence_after();
           kmajor_mma(tmem + L::kTmS, sk, q_of(g));     // S^T = K Q^T of the item's first query tile
@@ -352,8 +386,8 @@ __global__ void __launch_bounds__(512, 1)
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < 8; ++k)                 // dV += P_bar^T dO_i
-              umma_ts(tmem + L::kTmDV, tmem + L::pt_col(k), make_sdesc_sw128(sdo + k * 2048, L::kSubBytes, 1024),
-                      kIdAcc, (it > 0 || k > 0) ? 1u : 0u);
+              umma_ts_lh(tmem + L::kTmDV, tmem + L::pt_col(k), (sdo + k * (2048 >> 4)) | kLboMN, kHi, kIdAcc,
+                         (it > 0 || k > 0) ? 1u : 0u);
             umma_commit(pt_free);
             umma_commit(&do_empty[g % L::kDOStages]);   // dP_i and dV_i were the readers of dO_i
             if (it + 1 < w.n_it) {                      // S^T_{i+1}
@@ -366,18 +400,18 @@ __global__ void __launch_bounds__(512, 1)
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < 8; ++k)                 // dK += dS^T Q_i
-              umma_ts(tmem + L::kTmDK, tmem + L::dst_col(k), make_sdesc_sw128(sq + k * 2048, L::kSubBytes, 1024),
-                      kIdAcc, (it > 0 || k > 0) ? 1u : 0u);
+              umma_ts_lh(tmem + L::kTmDK, tmem + L::dst_col(k), (sq + k * (2048 >> 4)) | kLboMN, kHi, kIdAcc,
+                         (it > 0 || k > 0) ? 1u : 0u);
             if (!L::kWide && g > 0) {                   // the drain has read dQ of the previous step
               if (!(ok = mbar_wait(dq_free, (g - 1) & 1, wd))) break;
               tc_fence_after();
             }
 #pragma unroll
             for (int k = 0; k < 8; ++k)                 // dQ_i = dS K
-              umma_ss(tmem + L::kTmDQ, make_sdesc_sw128(sds + k * 2048, L::kSubBytes, 1024),
-                      make_sdesc_sw128(sk + k * 2048, L::kSubBytes, 1024), kIdDQ, k > 0 ? 1u : 0u);
+              umma_ss_lh(tmem + L::kTmDQ, ds_lo + k * (2048 >> 4), (sk + k * (2048 >> 4)) | kLboMN, kHi, kIdDQ,
+                         k > 0 ? 1u : 0u);
             umma_commit(dq_full);
-            umma_commit(&q_empty[g & 1]);
+            umma_commit(&q_empty[g % L::kQStages]);
             if (it + 1 < w.n_it) {                      // dP^T_{i+1}
               if (L::kWide) {                           // dQ_i shares the dP^T columns
                 if (!(ok = mbar_wait(dq_free, g & 1, wd))) break;
@@ -415,12 +449,12 @@ __global__ void __launch_bounds__(512, 1)
       const BwdItem w = bwd_item(p, item);
       const bool key_in = w.key0 + kr < p.N;
       for (int it = 0; it < w.n_it; ++it, ++g) {
-        const uint32_t st = g & 1;
+        const uint32_t st = g % L::kQStages;
         const int qt = w.i_start + it;
         const float* nlse = stats + st * 256 + 64 * half;
         const float* dd = stats + st * 256 + 128 + 64 * half;
         // q_full publishes this stage's LSE/D (written by the producer's lanes)
-        ok = __all_sync(0xffffffffu, mbar_wait(&q_full[st], (g >> 1) & 1, wd)) &&
+        ok = __all_sync(0xffffffffu, mbar_wait(&q_full[st], (g / L::kQStages) & 1, wd)) &&
              __all_sync(0xffffffffu, mbar_wait(s_full, g & 1, wd));
         if (!ok) break;
         tc_fence_after();

@@ -235,6 +235,43 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
   return d;
 }
 
+// The same descriptor as two 32-bit halves, for an issuing thread that must
+// spend as few instructions as possible per MMA: the low half holds the start
+// address and the leading byte offset, the high half the stride byte offset,
+// version and layout (shared by every operand with the same stride).
+// Advancing an operand is then one 32-bit add on its low half.
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo) {
+  return ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t sdesc_hi(uint32_t sbo) {
+  return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+
+// umma_ss / umma_ts with descriptors given as (low half, shared high half) and
+// the accumulate flag as a compile-time constant where the caller knows it.
+__device__ __forceinline__ void umma_ss_lh(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t.reg .b64 A, B;\n\t"
+      "setp.ne.b32 P, %5, 0;\n\t"
+      "mov.b64 A, {%1, %3};\n\t"
+      "mov.b64 B, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], A, B, %4, P;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_ts_lh(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t.reg .b64 B;\n\t"
+      "setp.ne.b32 P, %5, 0;\n\t"
+      "mov.b64 B, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], B, %4, P;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // A descriptor advanced by `bytes` along its start address (bits 0-13 hold
 // address >> 4; shared-memory addresses stay below 256 KB, so no carry
 // leaves the field).
