@@ -468,17 +468,29 @@ __global__ void __launch_bounds__(512, 1)
           tmem_ld_wait(r[1]);
           const bool diag = p.causal && qt == w.kv_tile;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int q = 2 * i;                       // query within this half
-            const uint64_t nl = *reinterpret_cast<const uint64_t*>(nlse + q);
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
-                                     __uint_as_float(r[i >> 4][(2 * i + 1) & 31])), c2, nl), x0, x1);
-            float p0 = ex2(x0), p1 = ex2(x1);
-            const int qg = 64 * half + q;              // query within the tile
-            if (!key_in || (diag && qg < kr)) p0 = 0.f;
-            if (!key_in || (diag && qg + 1 < kr)) p1 = 0.f;
-            pk[i] = pack_bf16(p0, p1);
+          for (int j = 0; j < 16; ++j) {               // 4 queries per shared-memory load of -LSE2
+            const float4 nl = *reinterpret_cast<const float4*>(nlse + 4 * j);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int i = 2 * j + h;                 // pair of queries 2i, 2i+1 of this half
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
+                                       __uint_as_float(r[i >> 4][(2 * i + 1) & 31])),
+                               c2, h ? f2_pack(nl.z, nl.w) : f2_pack(nl.x, nl.y)),
+                        x0, x1);
+              pk[i] = pack_bf16(ex2(x0), ex2(x1));
+            }
+          }
+          // masked keys (past N) and, on the diagonal tile, queries before the
+          // key: zero the packed halves (the warp takes this branch together)
+          if (__any_sync(0xffffffffu, !key_in || diag)) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int qg = 64 * half + 2 * i;        // query within the tile
+              const uint32_t lo = (!key_in || (diag && qg < kr)) ? 0u : 0x0000ffffu;
+              const uint32_t hi = (!key_in || (diag && qg + 1 < kr)) ? 0u : 0xffff0000u;
+              pk[i] &= lo | hi;
+            }
           }
         }
         if (!L::kWide && g > 0) {                      // dV of the previous step has read P_bar^T
@@ -509,14 +521,19 @@ __global__ void __launch_bounds__(512, 1)
           tmem_ld_wait(r[0]);
           tmem_ld_wait(r[1]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[i]));
-            const uint64_t dq2 = *reinterpret_cast<const uint64_t*>(dd + 2 * i);
-            const uint64_t dp2 = f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
-                                         __uint_as_float(r[i >> 4][(2 * i + 1) & 31]));
-            float y0, y1;
-            f2_unpack(f2_mul(f2_fma(dq2, f2_pack(-1.f, -1.f), dp2), f2_pack(pp.x, pp.y)), y0, y1);
-            dsw[i] = pack_bf16(y0, y1);
+          for (int j = 0; j < 16; ++j) {               // 4 queries per shared-memory load of D
+            const float4 d4 = *reinterpret_cast<const float4*>(dd + 4 * j);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int i = 2 * j + h;
+              const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[i]));
+              const uint64_t dq2 = h ? f2_pack(d4.z, d4.w) : f2_pack(d4.x, d4.y);
+              const uint64_t dp2 = f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
+                                           __uint_as_float(r[i >> 4][(2 * i + 1) & 31]));
+              float y0, y1;
+              f2_unpack(f2_mul(f2_fma(dq2, f2_pack(-1.f, -1.f), dp2), f2_pack(pp.x, pp.y)), y0, y1);
+              dsw[i] = pack_bf16(y0, y1);
+            }
           }
         }
         {
