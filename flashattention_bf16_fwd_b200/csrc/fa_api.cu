@@ -12,6 +12,7 @@
 #include "../../include/fa_b200.h"
 #include "fa_bwd.cuh"
 #include "fa_fwd.cuh"
+#include "fa_selftest.cuh"
 
 namespace fa {
 
@@ -328,6 +329,15 @@ const char* fa_status_string(int status) {
       return "fa_bwd_noalloc: fa_bwd_workspace_size() exceeds FA_BWD_NOALLOC_SCRATCH_BYTES (32 MiB)";
     default: return "unknown status";
   }
+}
+
+int fa_watchdog_selftest(unsigned timeout_us, void* stream) {
+  if (timeout_us < 1 || timeout_us > 1000000) return FA_ERR_ARG;
+  DeviceState* st = device_state();
+  if (!st) return FA_ERR_DEVICE;
+  const cudaError_t e = launch(fa_watchdog_selftest_kernel, dim3(1), dim3(64), 0, static_cast<cudaStream_t>(stream),
+                               st->dev_error, uint64_t(timeout_us) * 1000ull);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 int fa_check_device_error(void* stream) {

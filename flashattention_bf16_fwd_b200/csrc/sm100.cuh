@@ -80,13 +80,14 @@ struct Watchdog {
 // false (and marks the CTA aborted, and records kDevErrTimeout) when the wait
 // exceeds kWaitTimeoutNs, or when another role of the CTA already aborted.
 // The clock is read only every 1024 polls, so that each wait site stays small.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Watchdog& wd) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Watchdog& wd,
+                                          uint64_t timeout_ns = kWaitTimeoutNs) {
   uint32_t spins = 0;
   uint64_t deadline = 0;
   while (!mbar_try_wait(bar, parity)) {
     if ((++spins & 1023u) == 0) {
       const uint64_t now = globaltimer_ns();
-      if (deadline == 0) deadline = now + kWaitTimeoutNs;
+      if (deadline == 0) deadline = now + timeout_ns;
       if (*wd.abort || now > deadline) {
         if (!*wd.abort) atomicExch(wd.dev_error, kDevErrTimeout);
         *wd.abort = 1;

@@ -14,7 +14,7 @@ import torch
 
 __all__ = [
     "FAError", "LIB_PATH", "lib", "fa_fwd", "fa_fwd_ties", "fa_bwd", "fa_bwd_workspace_size",
-    "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc",
+    "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc", "fa_watchdog_selftest",
     "fa_status_string", "fa_check_device_error", "EXPORTED", "attention_fwd", "attention_bwd",
 ]
 
@@ -22,7 +22,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.
 
 FA_OK = 0
 EXPORTED = ("fa_fwd", "fa_fwd_ties", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
-            "fa_bwd_finish", "fa_bwd_noalloc", "fa_status_string", "fa_check_device_error")
+            "fa_bwd_finish", "fa_bwd_noalloc", "fa_watchdog_selftest", "fa_status_string",
+            "fa_check_device_error")
 
 
 class FAError(RuntimeError):
@@ -54,6 +55,8 @@ def _load() -> ctypes.CDLL:
     so.fa_bwd_finish.restype = i
     so.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
     so.fa_bwd_noalloc.restype = i
+    so.fa_watchdog_selftest.argtypes = [ctypes.c_uint, vp]
+    so.fa_watchdog_selftest.restype = i
     so.fa_status_string.argtypes = [i]
     so.fa_status_string.restype = ctypes.c_char_p
     so.fa_check_device_error.argtypes = [vp]
@@ -141,6 +144,10 @@ def fa_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, causal: bool, scale: float, 
     B, H, N, d = _shape(q)
     return lib.fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
                               _ptr(dv), B, H, N, d, int(causal), float(scale), _stream(stream))
+
+
+def fa_watchdog_selftest(timeout_us: int, stream=None) -> int:
+    return lib.fa_watchdog_selftest(int(timeout_us), _stream(stream))
 
 
 def fa_check_device_error(stream=None) -> int:

@@ -178,6 +178,19 @@ FA_API int fa_bwd_noalloc(const void* q, const void* k, const void* v,
 FA_API const char* fa_status_string(int status);
 
 /*
+ * fa_watchdog_selftest - test hook for the kernels' failure handling; the
+ * paper has no counterpart.  Launches one small kernel on `stream` whose
+ * bounded mbarrier wait (the same code every attention kernel uses) is made to
+ * expire after `timeout_us` microseconds (1 .. 1000000), while a second warp
+ * waits with the kernels' own limit and must leave on the CTA's abort mark.
+ * Nothing faults or hangs; the kernel returns, and the next
+ * fa_check_device_error() on that stream reports FA_ERR_TIMEOUT.
+ * Returns FA_OK, FA_ERR_ARG (timeout out of range), FA_ERR_DEVICE or
+ * FA_ERR_LAUNCH.
+ */
+FA_API int fa_watchdog_selftest(unsigned timeout_us, void* stream);
+
+/*
  * fa_check_device_error - synchronises `stream`, then reads and clears the
  * library's device error flag on the current device.  Returns FA_OK,
  * FA_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last check,

@@ -33,7 +33,8 @@ def declared_symbols():
 def test_header_declares_the_boundary():
     assert declared_symbols() == sorted(["fa_fwd", "fa_fwd_ties", "fa_bwd_workspace_size", "fa_bwd",
                                          "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish",
-                                         "fa_bwd_noalloc", "fa_status_string", "fa_check_device_error"])
+                                         "fa_bwd_noalloc", "fa_watchdog_selftest", "fa_status_string",
+                                         "fa_check_device_error"])
 
 
 def test_library_exports_every_declared_symbol(fa):
@@ -130,6 +131,12 @@ def test_valid_call_without_gpu_reports_device_error(fa):
     ws = fa.fa_bwd_workspace_size(1, 1, 128, 64)
     assert fa.lib.fa_bwd(A, A, A, A, A, A, A, A, A, A, ws, 1, 1, 128, 64, 1, 0.125, None) == FA_ERR_DEVICE
     assert fa.lib.fa_bwd_noalloc(A, A, A, A, A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, None) == FA_ERR_DEVICE
+    assert fa.lib.fa_watchdog_selftest(1000, None) == FA_ERR_DEVICE
+
+
+def test_watchdog_selftest_argument_errors(fa):
+    assert fa.lib.fa_watchdog_selftest(0, None) == FA_ERR_ARG
+    assert fa.lib.fa_watchdog_selftest(1000001, None) == FA_ERR_ARG
 
 
 def test_binding_rejects_cpu_tensors(fa):
