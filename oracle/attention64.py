@@ -27,6 +27,14 @@ What it computes, and where each step is stated:
   maximum included, is strictly below 1.  Reading taken here (the pages leave
   the amount open): m' = m + delta with delta = -ln(1 - 2^-8), so the maxima
   map to exactly 1 - 2^-8 = 0.99609375, the largest bf16 value below 1.
+* Variants of the fix, to measure which choices remove the bias (the pages
+  leave the amount of the shift open and trace the bias to P_bar = 1 in the
+  unnormalised output, same section): fix_mode 2 raises the shift by ln 2
+  (maxima -> 0.5, on the bf16 grid), fix_mode 3 by 1/16 (maxima ->
+  exp(-1/16) = 0.93941, off the grid: P_bar = 0.9375 there), and fix_mode 4
+  keeps the plain shift but divides by the sum of the rounded P_bar instead of
+  the unrounded P (a self-normalised output).  LSE is the unrounded
+  log-sum-exp in every mode.
 
 Parity pins for every function live in tests/test_oracle_pins.py (brute force,
 closed forms, invariants, finite differences, torch's bf16 cast).
@@ -36,13 +44,18 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "DELTA_LOG2", "DELTA_NAT", "bf16_round", "scores", "attention_fwd",
+    "DELTA_LOG2", "DELTA_NAT", "FIX_SHIFT_NAT", "SELF_NORMALISED_MODES", "bf16_round", "scores", "attention_fwd",
     "attention_bwd", "attention_fwd_bf16p", "tie_counts",
 ]
 
 # Shift added to m on repeated-max rows, in log2 units and in natural-log units.
 DELTA_LOG2 = -np.log2(1.0 - 2.0 ** -8)
 DELTA_NAT = -np.log(1.0 - 2.0 ** -8)
+
+# Shift (natural-log units) added on repeated-max rows for each fix_mode, and
+# the modes whose output is normalised by the sum of the rounded P_bar.
+FIX_SHIFT_NAT = {0: 0.0, 1: DELTA_NAT, 2: float(np.log(2.0)), 3: 1.0 / 16.0, 4: 0.0}
+SELF_NORMALISED_MODES = (4,)
 
 _BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
 
@@ -155,15 +168,17 @@ def attention_fwd_bf16p(q, k, v, causal: bool, scale: float, fix_mode: int,
     Per row i (one shift for the whole row):
       m_i    = max_j S_ij over visible keys,
       c_i    = #{j : S_ij == m_i}  (exact ties of the raw dot products),
-      m'_i   = m_i + DELTA_NAT if fix_mode == 1 and c_i >= 2, else m_i,
+      m'_i   = m_i + FIX_SHIFT_NAT[fix_mode] if c_i >= 2, else m_i,
       P_ij   = exp(S_ij - m'_i),          l_i = sum_j P_ij (unrounded),
       P_bar  = bf16(P) if round_p else P,
-      O_i    = (sum_j P_bar_ij V_j) / l_i,  LSE_i = m'_i + log l_i.
+      O_i    = (sum_j P_bar_ij V_j) / l_i   (fix_mode 4: / sum_j P_bar_ij),
+      LSE_i  = m'_i + log l_i.
     fix_mode 0 leaves the shift at the maximum, so repeated maxima give
-    P_bar == 1 exactly; fix_mode 1 maps them to 1 - 2^-8.
+    P_bar == 1 exactly; fix_mode 1 maps them to 1 - 2^-8, fix_mode 2 to 0.5,
+    fix_mode 3 to exp(-1/16); fix_mode 4 keeps them at 1 and self-normalises.
     """
-    if fix_mode not in (0, 1):
-        raise ValueError("fix_mode must be 0 or 1")
+    if fix_mode not in FIX_SHIFT_NAT:
+        raise ValueError("fix_mode must be 0, 1, 2, 3 or 4")
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, N, d = q.shape
     o = np.empty((B, H, N, v.shape[-1]))
@@ -175,11 +190,12 @@ def attention_fwd_bf16p(q, k, v, causal: bool, scale: float, fix_mode: int,
         ties = np.sum(raw == raw.max(axis=1, keepdims=True), axis=1, keepdims=True)
         s = scale * raw
         m = s.max(axis=1, keepdims=True)
-        shift = m + (DELTA_NAT if fix_mode == 1 else 0.0) * (ties >= 2)
+        shift = m + FIX_SHIFT_NAT[fix_mode] * (ties >= 2)
         p = np.exp(s - shift)
         l = p.sum(axis=1, keepdims=True)
         pbar = bf16_round(p) if round_p else p
-        o[b, h] = (pbar @ v[b, h]) / l
+        den = pbar.sum(axis=1, keepdims=True) if fix_mode in SELF_NORMALISED_MODES else l
+        o[b, h] = (pbar @ v[b, h]) / den
         lse[b, h] = shift[:, 0] + np.log(l[:, 0])
         if return_pbar:
             pbars[b, h] = pbar

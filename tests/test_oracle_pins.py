@@ -12,7 +12,11 @@ The pages print no worked example, so the oracle is pinned by
 * torch's CPU float32 -> bf16 cast for the bf16 rounding;
 * the fix's defining property ("Why Low-Precision Transformer Training Fails",
   mechanism 2): on repeated-max rows every P_bar, the maxima included, is
-  strictly below 1 (exactly 1 - 2^-8 at the maxima); without it they are 1.
+  strictly below 1 (exactly 1 - 2^-8 at the maxima); without it they are 1;
+* the fix variants: the maxima land on 0.5 (fix_mode 2) and on exp(-1/16),
+  0.9375 after rounding (fix_mode 3); the self-normalised mode (4) gives O = 1
+  exactly for V = 1, which the unrounded denominator does not; LSE is the
+  unrounded log-sum-exp in every mode.
 
 A mutation suite then plants plausible mistakes in a copy of the oracle's
 source and checks that each one trips at least one pin.
@@ -204,7 +208,7 @@ def emulation_pins(M):
     q, k, v = _rand(rng, 1, 2, 9, 4), _rand(rng, 1, 2, 9, 4), _rand(rng, 1, 2, 9, 4)
     k[0, 0, 7] = k[0, 0, 2]
     o, lse = M.attention_fwd(q, k, v, True, 0.6)
-    for fix in (0, 1):
+    for fix in (0, 1, 2, 3, 4):
         oe, le = M.attention_fwd_bf16p(q, k, v, True, 0.6, fix, round_p=False)
         if not (np.allclose(oe, o, atol=1e-13) and np.allclose(le, lse, atol=1e-13)):
             failed.append(f"unrounded_equals_exact_fix{fix}")
@@ -246,6 +250,36 @@ def emulation_pins(M):
     if not (np.array_equal(pb32.astype(np.float64), pb) and
             np.array_equal(torch.from_numpy(pb32).to(torch.bfloat16).float().numpy(), pb32)):
         failed.append("pbar_off_bf16_grid")
+    # E5 the variants of the fix: where each puts the maxima of a repeated-max
+    # row (unrounded, and after the bf16 rounding), and the self-normalised mode
+    q, k, v = _tie_inputs(rng)
+    ties = np.stack([np.asarray(brute_ties(q[0, h].tolist(), k[0, h].tolist(), True)) for h in range(2)])
+    for fix, top, top_bf16 in ((2, 0.5, 0.5), (3, float(np.exp(-1.0 / 16.0)), 0.9375)):
+        _, _, pu = M.attention_fwd_bf16p(q, k, v, True, 0.5, fix, round_p=False, return_pbar=True)
+        _, _, pr = M.attention_fwd_bf16p(q, k, v, True, 0.5, fix, return_pbar=True)
+        ok = True
+        for h in range(2):
+            for i in range(q.shape[2]):
+                ru, rr = pu[0, h, i, : i + 1], pr[0, h, i, : i + 1]
+                if ties[h, i] >= 2:
+                    ok &= abs(ru.max() - top) <= 1e-15 and np.sum(np.abs(ru - top) <= 1e-15) == ties[h, i]
+                    ok &= rr.max() == top_bf16 and np.all(ru < 1.0)
+                else:
+                    ok &= ru.max() == 1.0
+        if not ok:
+            failed.append(f"variant_maxima_fix{fix}")
+    # self-normalised: V = 1 gives O = 1 exactly, which the unrounded
+    # denominator does not; LSE stays the unrounded log-sum-exp in every mode
+    ones = np.ones_like(v)
+    o4, _ = M.attention_fwd_bf16p(q, k, ones, True, 0.5, 4)
+    o0, _ = M.attention_fwd_bf16p(q, k, ones, True, 0.5, 0)
+    if not (np.allclose(o4, 1.0, atol=1e-14, rtol=0) and not np.allclose(o0, 1.0, atol=1e-6, rtol=0)):
+        failed.append("self_normalised_ones")
+    _, lse_exact = M.attention_fwd(q, k, v, True, 0.5)
+    for fix in (0, 1, 2, 3, 4):
+        _, le = M.attention_fwd_bf16p(q, k, v, True, 0.5, fix)
+        if not np.allclose(le, lse_exact, atol=1e-13, rtol=0):
+            failed.append(f"lse_unrounded_fix{fix}")
     # E4 exact tie counts against brute force
     q, k, v = _tie_inputs(rng)
     for causal in (True, False):
@@ -324,6 +358,11 @@ MUTATIONS = [
     ("fix_wrong_delta", "DELTA_NAT = -np.log(1.0 - 2.0 ** -8)", "DELTA_NAT = -np.log(1.0 - 2.0 ** -6)"),
     ("emulation_skips_rounding", "pbar = bf16_round(p) if round_p else p", "pbar = p"),
     ("ties_ignore_mask", "s = np.where(vis, q[b, h] @ k[b, h].T, -np.inf)\n        out[b, h]", "s = q[b, h] @ k[b, h].T\n        out[b, h]"),
+    ("variant_shift_in_log2", "2: float(np.log(2.0))", "2: 1.0"),
+    ("variant_off_grid_value", "3: 1.0 / 16.0", "3: 1.0 / 8.0"),
+    ("self_normalised_unrounded_den", "den = pbar.sum(axis=1, keepdims=True) if", "den = l if"),
+    ("self_normalised_lse_from_pbar", "lse[b, h] = shift[:, 0] + np.log(l[:, 0])",
+     "lse[b, h] = shift[:, 0] + np.log(den[:, 0])"),
 ]
 
 
