@@ -156,7 +156,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   int rc = check_common(B, H, N, d, causal, scale);
   if (rc != FA_OK) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGN;
-  if (fix_mode != 0 && fix_mode != 1) return FA_ERR_FIXMODE;
+  if (fix_mode < 0 || fix_mode > 4) return FA_ERR_FIXMODE;
   DeviceState* st = device_state();
   if (!st) return FA_ERR_DEVICE;
   const int BH = B * H;
@@ -173,8 +173,13 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   prm.n_pairs = (N + 255) / 256;
   prm.causal = causal;
   prm.scale_log2 = float(double(scale) * 1.4426950408889634);
-  prm.delta_log2 = fix_mode ? float(kDeltaLog2) : 0.f;
-  prm.fix = fix_mode;
+  // shift on repeated-max rows per fix_mode, in base-2 units: 1 maps the
+  // maxima to 1 - 2^-8, 2 to 0.5, 3 to exp(-1/16); 0 and 4 keep the plain shift
+  const double delta = fix_mode == 1 ? kDeltaLog2 : fix_mode == 2 ? 1.0 : fix_mode == 3 ? 1.4426950408889634 / 16.0 : 0.0;
+  prm.delta_log2 = float(delta);
+  prm.fix_factor = float(std::exp2(-delta));
+  prm.fix = (fix_mode >= 1 && fix_mode <= 3) ? 1 : 0;
+  prm.self_norm = (fix_mode == 4) ? 1 : 0;
   const int n_items = prm.n_pairs * BH;
   const dim3 grid(unsigned(n_items < st->num_sms ? n_items : st->num_sms));
   const cudaError_t e =
@@ -319,7 +324,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_SHAPE: return "B, H or N < 1, or B*H*N*d >= 2^31";
     case FA_ERR_HEADDIM: return "head dimension d must be 64 or 128";
     case FA_ERR_ALIGN: return "a tensor base address is not 16-byte aligned";
-    case FA_ERR_FIXMODE: return "fix_mode must be 0 or 1";
+    case FA_ERR_FIXMODE: return "fix_mode must be 0, 1, 2, 3 or 4";
     case FA_ERR_WORKSPACE: return "workspace is NULL, misaligned or smaller than fa_bwd_workspace_size()";
     case FA_ERR_LAUNCH: return "the CUDA runtime refused a kernel launch";
     case FA_ERR_TIMEOUT: return "a kernel gave up on a bounded wait (device error flag set)";

@@ -38,7 +38,9 @@ struct FwdParams {
   int BH, N, n_pairs, causal;
   float scale_log2;     // scale * log2(e): S -> base-2 exponent domain
   float delta_log2;     // shift added to m on repeated-max rows (0 = fix off)
-  int fix;
+  float fix_factor;     // 2^-delta_log2: P at a repeated maximum (1 - 2^-8, 0.5 or exp(-1/16))
+  int fix;              // raise the shift on repeated-max rows
+  int self_norm;        // divide O by the sum of the rounded P_bar instead of the unrounded P
 };
 
 template <int D>
@@ -306,8 +308,8 @@ __global__ void __launch_bounds__(384, 1)
     const float sl2 = p.scale_log2;
     // 2^-delta: on a repeated-max row P is computed with the plain shift and
     // then multiplied by this, which is the same as raising m by delta; each
-    // maximum lands exactly on 1 - 2^-8.
-    const float kFixFactor = 0.99609375f;
+    // maximum lands on this value (1 - 2^-8 for fix_mode 1).
+    const float kFixFactor = p.fix_factor;
     uint32_t it_cnt = 0;   // softmax iterations done by this warpgroup
     bool ok = true;
 
@@ -324,6 +326,7 @@ __global__ void __launch_bounds__(384, 1)
       bool raised = false;  // the shift in use is ms + delta (fix active on this row)
       float l = 0.f;        // running sum of the unrounded P, relative to the shift in use
       bool ever_repeated = false;   // the running max occurred >= 2 times at some tile
+      float l_bar = 0.f;    // running sum of the rounded P_bar (self-normalised mode only)
 
       for (int j = 0; j < n_t; ++j) {
         const uint32_t ph = (it_cnt + j) & 1;
@@ -416,13 +419,20 @@ __global__ void __launch_bounds__(384, 1)
           if (!ok) break;
           tc_fence_after();
         }
+        float rs_bar = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]);
+          if (p.self_norm) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              rs_bar += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
+          }
           tmem_st16(t_p + c * 16, pk);
         }
+        l_bar = l_bar * alpha + rs_bar;
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
           const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll 1
@@ -460,7 +470,7 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t o[32];
         tmem_ld32(t_o + c * 32, o);
         tmem_ld_wait(o);
-        const float inv_l = 1.f / l;
+        const float inv_l = 1.f / (p.self_norm ? l_bar : l);
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           ow[c * 16 + i] = pack_bf16(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);

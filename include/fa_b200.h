@@ -58,7 +58,7 @@ typedef enum {
   FA_ERR_SHAPE = -2,     /* B, H or N < 1, or B*H*N*d too large               */
   FA_ERR_HEADDIM = -3,   /* d not in {64, 128}                                */
   FA_ERR_ALIGN = -4,     /* a tensor base is not 16-byte aligned              */
-  FA_ERR_FIXMODE = -5,   /* fix_mode not in {0, 1}                            */
+  FA_ERR_FIXMODE = -5,   /* fix_mode not in {0, 1, 2, 3, 4}                   */
   FA_ERR_WORKSPACE = -6, /* workspace NULL, misaligned or too small           */
   FA_ERR_LAUNCH = -7,    /* the CUDA runtime refused a launch                 */
   FA_ERR_TIMEOUT = -8,   /* a kernel's bounded wait expired (device flag)     */
@@ -75,7 +75,17 @@ typedef enum {
  *   o        out: bf16 [B,H,N,d], device.  O = (P_bar V) / l, rounded to bf16.
  *   lse      out: float32 [B,H,N], device.  LSE_i = log sum_j exp(S_ij).
  *   fix_mode    : 0 = plain safe softmax (shift = row max);
- *                 1 = repeated-max fix as described above.
+ *                 1 = repeated-max fix as described above (maxima -> 1 - 2^-8);
+ *                 the variants below measure which choices remove the bias
+ *                 (the pages leave the amount of the shift open):
+ *                 2 = the fix with the shift raised by 1 (base 2): maxima ->
+ *                     0.5, on the bf16 grid;
+ *                 3 = the fix with the shift raised by 1/16 (natural log):
+ *                     maxima -> exp(-1/16) = 0.93941, off the grid (P_bar
+ *                     0.9375 there);
+ *                 4 = plain shift, but O = (P_bar V) / sum_j P_bar_ij, the
+ *                     sum of the rounded P_bar (self-normalised).
+ *                 LSE is the unrounded log-sum-exp in every mode.
  * Returns FA_OK or a negative fa_status.
  */
 FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -86,10 +96,10 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* l
  * fa_fwd_ties - fa_fwd plus a per-row record of the repeated-max detector:
  *   ties out: int32 [B,H,N], device.  Bits 0-29: the number of visible keys
  *             whose FP32 score equals the row maximum of S (>= 2 means the
- *             fix applies to the final shift when fix_mode == 1).  Bit 30:
- *             set if the running maximum was repeated at any key tile, i.e.
- *             the detector fired at some point of the row (with fix_mode 1
- *             the shift was raised then).  Same kernel as fa_fwd; the extra
+ *             fix applies to the final shift when fix_mode is 1, 2 or 3).
+ *             Bit 30: set if the running maximum was repeated at any key
+ *             tile, i.e. the detector fired at some point of the row (with
+ *             fix_mode 1, 2 or 3 the shift was raised then).  Same kernel as fa_fwd; the extra
  *             store is one int per row.
  */
 FA_API int fa_fwd_ties(const void* q, const void* k, const void* v, void* o, float* lse,
