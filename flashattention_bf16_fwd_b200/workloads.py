@@ -11,6 +11,9 @@ Workloads (all causal, bf16, ``scale = 1/sqrt(d)``):
   their best key copied to a second visible position, so that the row maximum
   of S repeats ("Why Low-Precision Transformer Training Fails", mechanism 2:
   the fix targets rows whose maximum of S appears more than once).
+  ``structure="argmax_near"`` moves one element of each copy by one bf16 step,
+  against the row's query, so the copy scores just below the maximum: a near
+  tie whose probability still rounds to 1 (same page: P_bar exactly 1).
 * ``gpt2s``   B=8,  H=12, N=1024, d=64  - N(0,1) for Q, K, V, dO (GPT-2 small
   attention, the training runs of the same page's experiments section).
 * ``gpt2m``   B=8,  H=16, N=1024, d=64  - rank-4 keys K = U W plus an attention
@@ -45,7 +48,7 @@ class Workload:
     N: int
     d: int
     causal: bool = True
-    structure: str = "normal"       # normal | argmax_dup | lowrank_sink | key_dup
+    structure: str = "normal"       # normal | argmax_dup | argmax_near | lowrank_sink | key_dup
     frac: float = 0.0               # fraction of rows / keys touched by the structure
     rank: int = 4                   # rank of the keys for lowrank_sink
     sink_scale: float = 4.0         # sink key multiplier for lowrank_sink
@@ -83,11 +86,14 @@ def _to_bf16(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
 
 
-def _argmax_dup(rng, q16: torch.Tensor, k16: torch.Tensor, frac: float, causal: bool) -> torch.Tensor:
+def _argmax_dup(rng, q16: torch.Tensor, k16: torch.Tensor, frac: float, causal: bool,
+                near: bool = False) -> torch.Tensor:
     """Copy each chosen row's best visible key into a second visible position.
 
     Rows are visited in increasing order and always see the keys as modified so
-    far.  Row 0 of a causal head sees one key only and is never chosen.
+    far.  Row 0 of a causal head sees one key only and is never chosen.  With
+    ``near`` the copy's element at the query's smallest nonzero component moves
+    by one bf16 step in the direction that lowers the copy's score.
     """
     B, H, N, _ = q16.shape
     k = k16.clone()
@@ -104,6 +110,18 @@ def _argmax_dup(rng, q16: torch.Tensor, k16: torch.Tensor, frac: float, causal: 
                 others = [j for j in range(hi) if j != j_star]
                 j_dst = int(rng.choice(others))
                 k[b, h, j_dst] = k[b, h, j_star]
+                if near:
+                    qi = q16[b, h, i].to(torch.float64)
+                    ki = k[b, h, j_dst].to(torch.float64)
+                    ok = (qi != 0) & (ki != 0)
+                    if not bool(ok.any()):
+                        continue
+                    mag = torch.where(ok, qi.abs(), torch.full_like(qi, float("inf")))
+                    c = int(torch.argmin(mag))
+                    # bf16 is sign-magnitude: +1 on the bit pattern grows |k_c|,
+                    # -1 shrinks it; take the step that lowers q_c * k_c
+                    bits = k[b, h, j_dst, c:c + 1].view(torch.int16)
+                    bits += 1 if bool(qi[c] * ki[c] < 0) else -1
     return k
 
 
@@ -123,8 +141,8 @@ def make_inputs(w: Workload, seed: int = 0, with_grad: bool = True) -> dict:
     else:
         k = _to_bf16(rng.standard_normal(shape, dtype=np.float32))
     v = _to_bf16(rng.standard_normal(shape, dtype=np.float32))
-    if w.structure == "argmax_dup":
-        k = _argmax_dup(rng, q, k, w.frac, w.causal)
+    if w.structure in ("argmax_dup", "argmax_near"):
+        k = _argmax_dup(rng, q, k, w.frac, w.causal, near=(w.structure == "argmax_near"))
     elif w.structure == "key_dup":
         n_dup = int(round(w.frac * w.N))
         for b in range(w.B):

@@ -35,6 +35,10 @@ What it computes, and where each step is stated:
   keeps the plain shift but divides by the sum of the rounded P_bar instead of
   the unrounded P (a self-normalised output).  LSE is the unrounded
   log-sum-exp in every mode.
+* A near-tie detector (fix_mode 5), after the same section's statement that
+  the bias comes from probabilities of exactly 1: the shift is raised by
+  delta when at least two entries of the row have P_bar == 1 under the plain
+  shift (their P rounds to 1 in bf16), not only when S ties exactly.
 
 Parity pins for every function live in tests/test_oracle_pins.py (brute force,
 closed forms, invariants, finite differences, torch's bf16 cast).
@@ -44,8 +48,8 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "DELTA_LOG2", "DELTA_NAT", "FIX_SHIFT_NAT", "SELF_NORMALISED_MODES", "bf16_round", "scores", "attention_fwd",
-    "attention_bwd", "attention_fwd_bf16p", "tie_counts",
+    "DELTA_LOG2", "DELTA_NAT", "FIX_SHIFT_NAT", "SELF_NORMALISED_MODES", "NEAR_TIE_MODES", "bf16_round", "scores", "attention_fwd",
+    "attention_bwd", "attention_fwd_bf16p", "tie_counts", "near_tie_counts",
 ]
 
 # Shift added to m on repeated-max rows, in log2 units and in natural-log units.
@@ -54,7 +58,8 @@ DELTA_NAT = -np.log(1.0 - 2.0 ** -8)
 
 # Shift (natural-log units) added on repeated-max rows for each fix_mode, and
 # the modes whose output is normalised by the sum of the rounded P_bar.
-FIX_SHIFT_NAT = {0: 0.0, 1: DELTA_NAT, 2: float(np.log(2.0)), 3: 1.0 / 16.0, 4: 0.0}
+FIX_SHIFT_NAT = {0: 0.0, 1: DELTA_NAT, 2: float(np.log(2.0)), 3: 1.0 / 16.0, 4: 0.0, 5: DELTA_NAT}
+NEAR_TIE_MODES = (5,)
 SELF_NORMALISED_MODES = (4,)
 
 _BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
@@ -161,6 +166,19 @@ def tie_counts(q, k, causal: bool) -> np.ndarray:
     return out
 
 
+def near_tie_counts(q, k, causal: bool, scale: float) -> np.ndarray:
+    """#{j visible : bf16(exp(scale * (S_ij - max_j S_ij))) == 1} per row."""
+    q, k = _f64(q), _f64(k)
+    B, H, N, _ = q.shape
+    out = np.zeros((B, H, N), dtype=np.int64)
+    vis = _mask(N, causal)
+    for b, h in _heads(q):
+        s = np.where(vis, scale * (q[b, h] @ k[b, h].T), -np.inf)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        out[b, h] = np.sum(bf16_round(p) == 1.0, axis=1)
+    return out
+
+
 def attention_fwd_bf16p(q, k, v, causal: bool, scale: float, fix_mode: int,
                         round_p: bool = True, return_pbar: bool = False):
     """Attention with the safe-softmax shift, BF16-rounded P_bar and the fix.
@@ -168,17 +186,19 @@ def attention_fwd_bf16p(q, k, v, causal: bool, scale: float, fix_mode: int,
     Per row i (one shift for the whole row):
       m_i    = max_j S_ij over visible keys,
       c_i    = #{j : S_ij == m_i}  (exact ties of the raw dot products),
-      m'_i   = m_i + FIX_SHIFT_NAT[fix_mode] if c_i >= 2, else m_i,
+      m'_i   = m_i + FIX_SHIFT_NAT[fix_mode] if c_i >= 2, else m_i
+               (fix_mode 5 counts c_i as the entries with bf16(exp(S_ij - m_i)) == 1),
       P_ij   = exp(S_ij - m'_i),          l_i = sum_j P_ij (unrounded),
       P_bar  = bf16(P) if round_p else P,
       O_i    = (sum_j P_bar_ij V_j) / l_i   (fix_mode 4: / sum_j P_bar_ij),
       LSE_i  = m'_i + log l_i.
     fix_mode 0 leaves the shift at the maximum, so repeated maxima give
     P_bar == 1 exactly; fix_mode 1 maps them to 1 - 2^-8, fix_mode 2 to 0.5,
-    fix_mode 3 to exp(-1/16); fix_mode 4 keeps them at 1 and self-normalises.
+    fix_mode 3 to exp(-1/16); fix_mode 4 keeps them at 1 and self-normalises;
+    fix_mode 5 is fix_mode 1 triggered by near ties.
     """
     if fix_mode not in FIX_SHIFT_NAT:
-        raise ValueError("fix_mode must be 0, 1, 2, 3 or 4")
+        raise ValueError("fix_mode must be 0, 1, 2, 3, 4 or 5")
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, N, d = q.shape
     o = np.empty((B, H, N, v.shape[-1]))
@@ -187,9 +207,12 @@ def attention_fwd_bf16p(q, k, v, causal: bool, scale: float, fix_mode: int,
     vis = _mask(N, causal)
     for b, h in _heads(q):
         raw = np.where(vis, q[b, h] @ k[b, h].T, -np.inf)
-        ties = np.sum(raw == raw.max(axis=1, keepdims=True), axis=1, keepdims=True)
         s = scale * raw
         m = s.max(axis=1, keepdims=True)
+        if fix_mode in NEAR_TIE_MODES:
+            ties = np.sum(bf16_round(np.exp(s - m)) == 1.0, axis=1, keepdims=True)
+        else:
+            ties = np.sum(raw == raw.max(axis=1, keepdims=True), axis=1, keepdims=True)
         shift = m + FIX_SHIFT_NAT[fix_mode] * (ties >= 2)
         p = np.exp(s - shift)
         l = p.sum(axis=1, keepdims=True)

@@ -16,7 +16,10 @@ The pages print no worked example, so the oracle is pinned by
 * the fix variants: the maxima land on 0.5 (fix_mode 2) and on exp(-1/16),
   0.9375 after rounding (fix_mode 3); the self-normalised mode (4) gives O = 1
   exactly for V = 1, which the unrounded denominator does not; LSE is the
-  unrounded log-sum-exp in every mode.
+  unrounded log-sum-exp in every mode;
+* the near-tie detector (fix_mode 5): counts against scalar loops with
+  math.exp and torch's bf16 cast on inputs with near ties but no exact ones,
+  and every P_bar below 1 on the rows it raises.
 
 A mutation suite then plants plausible mistakes in a copy of the oracle's
 source and checks that each one trips at least one pin.
@@ -280,6 +283,38 @@ def emulation_pins(M):
         _, le = M.attention_fwd_bf16p(q, k, v, True, 0.5, fix)
         if not np.allclose(le, lse_exact, atol=1e-13, rtol=0):
             failed.append(f"lse_unrounded_fix{fix}")
+    # E6 near ties: brute-force count (math.exp, torch's bf16 cast) and the
+    # defining property of fix_mode 5 on the rows it raises
+    from flashattention_bf16_fwd_b200.workloads import WORKLOADS as _W, make_inputs as _mk
+    x = _mk(_W["tiny"].with_shape(H=2, N=24, d=8, structure="argmax_near", frac=0.5), seed=7, with_grad=False)
+    qn, kn, vn = (x[n].double().numpy() for n in ("q", "k", "v"))
+    sc = x["scale"]
+    brute = np.zeros((1, 2, 24), dtype=np.int64)
+    exact_rep = np.zeros((1, 2, 24), dtype=bool)
+    for h in range(2):
+        for i in range(24):
+            row = [sc * sum(qn[0, h, i, c] * kn[0, h, j, c] for c in range(8)) for j in range(i + 1)]
+            mx = max(row)
+            pr = torch.tensor([math.exp(r - mx) for r in row], dtype=torch.float64)
+            brute[0, h, i] = int((pr.float().to(torch.bfloat16).float() == 1.0).sum())
+            exact_rep[0, h, i] = sum(r == mx for r in row) >= 2
+    near = M.near_tie_counts(qn, kn, True, sc)
+    if not np.array_equal(near, brute):
+        failed.append("near_tie_counts")
+    if not np.any((brute >= 2) & ~exact_rep):
+        failed.append("no_near_only_rows_in_fixture")
+    _, _, p5 = M.attention_fwd_bf16p(qn, kn, vn, True, sc, 5, return_pbar=True)
+    _, _, p0 = M.attention_fwd_bf16p(qn, kn, vn, True, sc, 0, return_pbar=True)
+    ok = True
+    for h in range(2):
+        for i in range(24):
+            r5, r0 = p5[0, h, i, : i + 1], p0[0, h, i, : i + 1]
+            if brute[0, h, i] >= 2:
+                ok &= bool(np.all(r5 < 1.0)) and np.sum(r0 == 1.0) == brute[0, h, i]
+            else:
+                ok &= np.array_equal(r5, r0)
+    if not ok:
+        failed.append("near_tie_fix_property")
     # E4 exact tie counts against brute force
     q, k, v = _tie_inputs(rng)
     for causal in (True, False):
@@ -361,6 +396,10 @@ MUTATIONS = [
     ("variant_shift_in_log2", "2: float(np.log(2.0))", "2: 1.0"),
     ("variant_off_grid_value", "3: 1.0 / 16.0", "3: 1.0 / 8.0"),
     ("self_normalised_unrounded_den", "den = pbar.sum(axis=1, keepdims=True) if", "den = l if"),
+    ("near_ties_count_exact_ties", "ties = np.sum(bf16_round(np.exp(s - m)) == 1.0, axis=1, keepdims=True)",
+     "ties = np.sum(raw == raw.max(axis=1, keepdims=True), axis=1, keepdims=True)"),
+    ("near_tie_no_shift", "4: 0.0, 5: DELTA_NAT}", "4: 0.0, 5: 0.0}"),
+    ("near_tie_threshold_off", "out[b, h] = np.sum(bf16_round(p) == 1.0, axis=1)", "out[b, h] = np.sum(p == 1.0, axis=1)"),
     ("self_normalised_lse_from_pbar", "lse[b, h] = shift[:, 0] + np.log(l[:, 0])",
      "lse[b, h] = shift[:, 0] + np.log(den[:, 0])"),
 ]
