@@ -61,16 +61,24 @@ DeviceState* device_state() {
     if (cudaGetSymbolAddress(&addr, g_dev_error) != cudaSuccess) return;
     st->dev_error = static_cast<int*>(addr);
     bool ok = true;
-    ok &= cudaFuncSetAttribute(fa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    ok &= cudaFuncSetAttribute(fa_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                FwdLayout<64>::kAlloc) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    ok &= cudaFuncSetAttribute(fa_fwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdLayout<128>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(fa_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdLayout<64>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(fa_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                FwdLayout<128>::kAlloc) == cudaSuccess;
     // The forward kernel moves registers between warpgroups with setmaxnreg;
     // the split assumes exactly kLaunchRegs registers per thread at launch.
     cudaFuncAttributes fattr{};
-    ok &= cudaFuncGetAttributes(&fattr, fa_fwd_kernel<64>) == cudaSuccess &&
+    ok &= cudaFuncGetAttributes(&fattr, fa_fwd_kernel<64, false>) == cudaSuccess &&
           fattr.numRegs == FwdLayout<64>::kLaunchRegs;
-    ok &= cudaFuncGetAttributes(&fattr, fa_fwd_kernel<128>) == cudaSuccess &&
+    ok &= cudaFuncGetAttributes(&fattr, fa_fwd_kernel<128, false>) == cudaSuccess &&
+          fattr.numRegs == FwdLayout<128>::kLaunchRegs;
+    ok &= cudaFuncGetAttributes(&fattr, fa_fwd_kernel<64, true>) == cudaSuccess &&
+          fattr.numRegs == FwdLayout<64>::kLaunchRegs;
+    ok &= cudaFuncGetAttributes(&fattr, fa_fwd_kernel<128, true>) == cudaSuccess &&
           fattr.numRegs == FwdLayout<128>::kLaunchRegs;
     ok &= cudaFuncGetAttributes(&fattr, fa_bwd_kernel<64>) == cudaSuccess &&
           fattr.numRegs == BwdLayout<64>::kLaunchRegs;
@@ -156,7 +164,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   int rc = check_common(B, H, N, d, causal, scale);
   if (rc != FA_OK) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGN;
-  if (fix_mode < 0 || fix_mode > 4) return FA_ERR_FIXMODE;
+  if (fix_mode < 0 || fix_mode > 5) return FA_ERR_FIXMODE;
   DeviceState* st = device_state();
   if (!st) return FA_ERR_DEVICE;
   const int BH = B * H;
@@ -173,20 +181,24 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   prm.n_pairs = (N + 255) / 256;
   prm.causal = causal;
   prm.scale_log2 = float(double(scale) * 1.4426950408889634);
-  // shift on repeated-max rows per fix_mode, in base-2 units: 1 maps the
+  // shift on repeated-max rows per fix_mode, in base-2 units: 1 and 5 map the
   // maxima to 1 - 2^-8, 2 to 0.5, 3 to exp(-1/16); 0 and 4 keep the plain shift
-  const double delta = fix_mode == 1 ? kDeltaLog2 : fix_mode == 2 ? 1.0 : fix_mode == 3 ? 1.4426950408889634 / 16.0 : 0.0;
+  const double delta = (fix_mode == 1 || fix_mode == 5) ? kDeltaLog2
+                       : fix_mode == 2                  ? 1.0
+                       : fix_mode == 3                  ? 1.4426950408889634 / 16.0
+                                                        : 0.0;
   prm.delta_log2 = float(delta);
   prm.fix_factor = float(std::exp2(-delta));
-  prm.fix = (fix_mode >= 1 && fix_mode <= 3) ? 1 : 0;
+  prm.fix = (fix_mode == 1 || fix_mode == 2 || fix_mode == 3 || fix_mode == 5) ? 1 : 0;
   prm.self_norm = (fix_mode == 4) ? 1 : 0;
+  prm.near = (fix_mode == 5) ? 1 : 0;
   const int n_items = prm.n_pairs * BH;
   const dim3 grid(unsigned(n_items < st->num_sms ? n_items : st->num_sms));
-  const cudaError_t e =
-      (d == 64) ? launch(fa_fwd_kernel<64>, grid, dim3(FwdLayout<64>::kThreads), FwdLayout<64>::kAlloc, stream, mq, mk,
-                         mv, prm)
-                : launch(fa_fwd_kernel<128>, grid, dim3(FwdLayout<128>::kThreads), FwdLayout<128>::kAlloc, stream, mq,
-                         mk, mv, prm);
+  const bool variants = fix_mode >= 4;   // self-normalised or near-tie code
+  auto kern = (d == 64) ? (variants ? fa_fwd_kernel<64, true> : fa_fwd_kernel<64, false>)
+                        : (variants ? fa_fwd_kernel<128, true> : fa_fwd_kernel<128, false>);
+  const int smem = (d == 64) ? FwdLayout<64>::kAlloc : FwdLayout<128>::kAlloc;
+  const cudaError_t e = launch(kern, grid, dim3(FwdLayout<64>::kThreads), smem, stream, mq, mk, mv, prm);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
@@ -324,7 +336,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_SHAPE: return "B, H or N < 1, or B*H*N*d >= 2^31";
     case FA_ERR_HEADDIM: return "head dimension d must be 64 or 128";
     case FA_ERR_ALIGN: return "a tensor base address is not 16-byte aligned";
-    case FA_ERR_FIXMODE: return "fix_mode must be 0, 1, 2, 3 or 4";
+    case FA_ERR_FIXMODE: return "fix_mode must be 0, 1, 2, 3, 4 or 5";
     case FA_ERR_WORKSPACE: return "workspace is NULL, misaligned or smaller than fa_bwd_workspace_size()";
     case FA_ERR_LAUNCH: return "the CUDA runtime refused a kernel launch";
     case FA_ERR_TIMEOUT: return "a kernel gave up on a bounded wait (device error flag set)";

@@ -41,6 +41,7 @@ struct FwdParams {
   float fix_factor;     // 2^-delta_log2: P at a repeated maximum (1 - 2^-8, 0.5 or exp(-1/16))
   int fix;              // raise the shift on repeated-max rows
   int self_norm;        // divide O by the sum of the rounded P_bar instead of the unrounded P
+  int near;             // detect near ties (P rounds to bf16 1.0) instead of exact ties of S
 };
 
 template <int D>
@@ -89,7 +90,9 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
   return it;
 }
 
-template <int D>
+// kVariants: compiled with the code of fix_mode 4 (self-normalised) and 5
+// (near ties); the other instantiation, used for fix_mode 0-3, leaves it out.
+template <int D, bool kVariants>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -327,6 +330,7 @@ __global__ void __launch_bounds__(384, 1)
       float l = 0.f;        // running sum of the unrounded P, relative to the shift in use
       bool ever_repeated = false;   // the running max occurred >= 2 times at some tile
       float l_bar = 0.f;    // running sum of the rounded P_bar (self-normalised mode only)
+      int cnt_near = 0;     // entries whose P rounds to 1 under the current shift (near-tie mode)
 
       for (int j = 0; j < n_t; ++j) {
         const uint32_t ph = (it_cnt + j) & 1;
@@ -381,8 +385,19 @@ __global__ void __launch_bounds__(384, 1)
         const int ct = (mt == kNegInf) ? 0 : int(ea + eb);
         int c_new = (m == m_new ? cnt : 0) + (mt == m_new ? ct : 0);
         if (m_new == kNegInf) c_new = 0;
-        ever_repeated |= (c_new >= 2);
-        const bool raise = p.fix && c_new >= 2;
+        // near-tie mode: entries of this tile whose P (plain shift) rounds to
+        // bf16 1.0, i.e. P >= 1 - 2^-9; earlier tiles' count stands while the
+        // shift has not moved
+        int cn_new = 0;
+        if (kVariants && p.near) {
+          int cn = 0;
+#pragma unroll
+          for (int i = 0; i < 128; ++i) cn += (s[i] >= 0.998046875f) ? 1 : 0;
+          cn_new = (m == m_new ? cnt_near : 0) + cn;
+        }
+        const int det = (kVariants && p.near) ? cn_new : c_new;
+        ever_repeated |= (det >= 2);
+        const bool raise = p.fix && det >= 2;
         f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), ea, eb);
         float rs = ea + eb;
         if (__any_sync(0xffffffffu, raise)) {
@@ -425,7 +440,7 @@ __global__ void __launch_bounds__(384, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]);
-          if (p.self_norm) {
+          if (kVariants && p.self_norm) {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               rs_bar += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
@@ -455,6 +470,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive(&p_full[t]);
         m = m_new;
         cnt = c_new;
+        cnt_near = cn_new;
         ms = ms_new;
         raised = raise;
       }
@@ -470,7 +486,7 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t o[32];
         tmem_ld32(t_o + c * 32, o);
         tmem_ld_wait(o);
-        const float inv_l = 1.f / (p.self_norm ? l_bar : l);
+        const float inv_l = 1.f / ((kVariants && p.self_norm) ? l_bar : l);
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           ow[c * 16 + i] = pack_bf16(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);

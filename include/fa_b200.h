@@ -58,7 +58,7 @@ typedef enum {
   FA_ERR_SHAPE = -2,     /* B, H or N < 1, or B*H*N*d too large               */
   FA_ERR_HEADDIM = -3,   /* d not in {64, 128}                                */
   FA_ERR_ALIGN = -4,     /* a tensor base is not 16-byte aligned              */
-  FA_ERR_FIXMODE = -5,   /* fix_mode not in {0, 1, 2, 3, 4}                   */
+  FA_ERR_FIXMODE = -5,   /* fix_mode not in {0, 1, 2, 3, 4, 5}                */
   FA_ERR_WORKSPACE = -6, /* workspace NULL, misaligned or too small           */
   FA_ERR_LAUNCH = -7,    /* the CUDA runtime refused a launch                 */
   FA_ERR_TIMEOUT = -8,   /* a kernel's bounded wait expired (device flag)     */
@@ -84,7 +84,12 @@ typedef enum {
  *                     maxima -> exp(-1/16) = 0.93941, off the grid (P_bar
  *                     0.9375 there);
  *                 4 = plain shift, but O = (P_bar V) / sum_j P_bar_ij, the
- *                     sum of the rounded P_bar (self-normalised).
+ *                     sum of the rounded P_bar (self-normalised);
+ *                 5 = fix_mode 1 triggered by near ties: two or more entries
+ *                     whose P (plain shift) rounds to bf16 1.0, i.e.
+ *                     P >= 1 - 2^-9.  Counted per key tile under the shift in
+ *                     use; a count from earlier tiles is dropped when the row
+ *                     maximum moves.
  *                 LSE is the unrounded log-sum-exp in every mode.
  * Returns FA_OK or a negative fa_status.
  */
@@ -97,9 +102,10 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* l
  *   ties out: int32 [B,H,N], device.  Bits 0-29: the number of visible keys
  *             whose FP32 score equals the row maximum of S (>= 2 means the
  *             fix applies to the final shift when fix_mode is 1, 2 or 3).
- *             Bit 30: set if the running maximum was repeated at any key
- *             tile, i.e. the detector fired at some point of the row (with
- *             fix_mode 1, 2 or 3 the shift was raised then).  Same kernel as fa_fwd; the extra
+ *             Bit 30: set if the detector fired at some key tile: the
+ *             running maximum was repeated (fix_mode 0-4), or two or more
+ *             entries rounded to 1 (fix_mode 5); with fix_mode 1, 2, 3 or 5
+ *             the shift was raised then.  Same kernel as fa_fwd; the extra
  *             store is one int per row.
  */
 FA_API int fa_fwd_ties(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -82,7 +82,7 @@ def test_fwd_argument_errors(fa):
     assert fwd(fa, scale=float("inf")) == FA_ERR_ARG
     assert fwd(fa, k=MIS) == FA_ERR_ALIGN
     assert fwd(fa, o=MIS) == FA_ERR_ALIGN
-    assert fwd(fa, fix=5) == FA_ERR_FIXMODE
+    assert fwd(fa, fix=6) == FA_ERR_FIXMODE
     assert fwd(fa, fix=-1) == FA_ERR_FIXMODE
     assert fa.lib.fa_fwd_ties(A, A, A, A, A, None, 1, 1, 128, 64, 1, 0.125, 1, None) == FA_ERR_NULL
 

@@ -1,8 +1,9 @@
-"""GPU parity of the fix variants (fix_mode 2, 3, 4) and the bias sweep.
+"""GPU parity of the fix variants (fix_mode 2-5) and the bias sweep.
 
 fix_mode 2 and 3 raise the shift on repeated-max rows by 1 (base 2) and by
 1/16 (natural log), so the maxima land on 0.5 and on exp(-1/16); fix_mode 4
-keeps the plain shift and divides by the sum of the rounded P_bar.  All of
+keeps the plain shift and divides by the sum of the rounded P_bar; fix_mode 5
+is fix_mode 1 triggered by near ties (P rounds to bf16 1.0).  All of
 them compute the same attention up to rounding, so the exact FP64 oracle and
 the tolerances of the parity tests apply unchanged; the emulating oracle
 (one shift per row, bf16 P_bar) of each mode is checked as well.
@@ -13,7 +14,7 @@ import torch
 
 from flashattention_bf16_fwd_b200.stats import bias_stats, lse_rel_err
 from flashattention_bf16_fwd_b200.workloads import WORKLOADS, Workload, make_inputs
-from oracle import attention_fwd, attention_fwd_bf16p, tie_counts
+from oracle import attention_fwd, attention_fwd_bf16p, near_tie_counts, tie_counts
 
 pytestmark = pytest.mark.gpu
 
@@ -42,7 +43,7 @@ SHAPES = [(1, 2, 127, 64, 1), (1, 2, 1000, 64, 1), (1, 1, 200, 128, 1), (1, 2, 3
 
 
 @pytest.mark.parametrize("B,H,N,d,causal", SHAPES, ids=[f"B{b}H{h}N{n}d{d}{'c' if c else 'f'}" for b, h, n, d, c in SHAPES])
-@pytest.mark.parametrize("fix_mode", [2, 3, 4])
+@pytest.mark.parametrize("fix_mode", [2, 3, 4, 5])
 def test_variant_parity(fa, B, H, N, d, causal, fix_mode):
     x = make_inputs(Workload("shape", B, H, N, d, causal=bool(causal)), seed=N + d, with_grad=False)
     o, lse, _ = fwd(fa, x, fix_mode)
@@ -71,6 +72,44 @@ def test_variant_on_repeated_maxima(fa, fix_mode):
         assert np.array_equal(o[quiet], o0[quiet])
 
 
+def test_near_tie_detector(fa):
+    """fix_mode 5 on inputs with near ties and no exact ties: the detector
+    fires where the oracle counts two or more entries rounding to 1 (one key
+    tile, so the kernel's per-tile count is the whole row's), the exact
+    detector does not fire, and rows left alone run fix_mode 0's arithmetic."""
+    x = make_inputs(WORKLOADS["tiny"].with_shape(structure="argmax_near"), seed=0, with_grad=False)
+    o5, lse5, t5 = fwd(fa, x, 5)
+    o1, _, t1 = fwd(fa, x, 1)
+    o0, lse0, _ = fwd(fa, x, 0)
+    near = near_tie_counts(x["q"], x["k"], True, x["scale"]) >= 2
+    assert near.sum() > 50
+    fired5 = ((t5 >> 30) & 1) == 1
+    assert np.mean(fired5 == near) >= 0.99
+    # the copies differ from the maximum in FP64 but a few still tie after the
+    # tensor core's FP32 accumulation: the exact detector fires on those only
+    assert np.mean(((t1 >> 30) & 1) == 1) <= 0.05
+    assert np.array_equal(o5[~fired5], o0[~fired5]) and np.array_equal(lse5[~fired5], lse0[~fired5])
+    oe, le = attention_fwd_bf16p(x["q"], x["k"], x["v"], True, x["scale"], 5)
+    assert np.abs(o5 - oe).max() <= O_ATOL
+    assert lse_rel_err(lse5, le) <= LSE_RTOL
+    o_ref, _ = attention_fwd(x["q"], x["k"], x["v"], True, x["scale"])
+    assert np.abs(o5 - o_ref).max() <= O_ATOL
+
+
+def test_near_tie_bias(fa):
+    """Bias on near-tie rows (no exact ties) for fix_mode 0, 1, 4 and 5 (printed)."""
+    x = make_inputs(WORKLOADS["tiny"].with_shape(B=2, H=4, N=1024, structure="argmax_near"), seed=3,
+                    with_grad=False)
+    o_ref, _ = attention_fwd(x["q"], x["k"], x["v"], True, x["scale"])
+    near = near_tie_counts(x["q"], x["k"], True, x["scale"]) >= 2
+    assert near.sum() > 500
+    for mode in (0, 1, 4, 5):
+        o, _, _ = fwd(fa, x, mode)
+        s = bias_stats(o, o_ref, near)
+        print(f"near-tie rows ({s['rows']}), fix_mode {mode}: z_mean {s['z_mean']:+.2f}  "
+              f"z_aligned {s['z_aligned']:+.2f}  aligned_mean/mean|O| {s['aligned_mean'] / s['mean_abs_ref']:+.3e}")
+
+
 def test_self_normalised_output_of_ones(fa):
     """With V = 1 every row of O is a sum of weights that add up to 1 exactly
     in fix_mode 4; with the unrounded denominator (fix_mode 0) they do not."""
@@ -90,7 +129,7 @@ def test_bias_sweep_over_fix_modes(fa):
     rep = tie_counts(x["q"], x["k"], True) >= 2
     assert rep.sum() > 1000
     rows = {}
-    for mode in range(5):
+    for mode in range(6):
         o, _, _ = fwd(fa, x, mode)
         s = bias_stats(o, o_ref, rep)
         rows[mode] = s
