@@ -35,6 +35,11 @@ What it computes, and where each step is stated:
   keeps the plain shift but divides by the sum of the rounded P_bar instead of
   the unrounded P (a self-normalised output).  LSE is the unrounded
   log-sum-exp in every mode.
+* Grouped-query attention (GQA/MQA head layouts, the Llama 2 family the
+  chibakuma.com page names): H_q query heads share H_kv key/value heads,
+  query head h reading key/value head h // (H_q / H_kv).  The forward is the
+  definition above with K and V repeated over each group; the gradients of a
+  shared K or V head are the sums over its group.
 * A near-tie detector (fix_mode 5), after the same section's statement that
   the bias comes from probabilities of exactly 1: the shift is raised by
   delta when at least two entries of the row have P_bar == 1 under the plain
@@ -49,7 +54,7 @@ import numpy as np
 
 __all__ = [
     "DELTA_LOG2", "DELTA_NAT", "FIX_SHIFT_NAT", "SELF_NORMALISED_MODES", "NEAR_TIE_MODES", "bf16_round", "scores", "attention_fwd",
-    "attention_bwd", "attention_fwd_bf16p", "tie_counts", "near_tie_counts",
+    "attention_bwd", "attention_fwd_bf16p", "tie_counts", "near_tie_counts", "gqa_expand", "gqa_reduce",
 ]
 
 # Shift added to m on repeated-max rows, in log2 units and in natural-log units.
@@ -164,6 +169,18 @@ def tie_counts(q, k, causal: bool) -> np.ndarray:
         s = np.where(vis, q[b, h] @ k[b, h].T, -np.inf)
         out[b, h] = np.sum(s == s.max(axis=1, keepdims=True), axis=1)
     return out
+
+
+def gqa_expand(x, group: int) -> np.ndarray:
+    """[B, H_kv, N, d] -> [B, H_kv * group, N, d]: each head repeated for its group."""
+    return np.repeat(_f64(x), group, axis=1)
+
+
+def gqa_reduce(x, group: int) -> np.ndarray:
+    """[B, H_kv * group, N, d] -> [B, H_kv, N, d]: the sum over each group."""
+    x = _f64(x)
+    B, H, N, d = x.shape
+    return x.reshape(B, H // group, group, N, d).sum(axis=2)
 
 
 def near_tie_counts(q, k, causal: bool, scale: float) -> np.ndarray:

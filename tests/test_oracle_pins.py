@@ -17,6 +17,8 @@ The pages print no worked example, so the oracle is pinned by
   0.9375 after rounding (fix_mode 3); the self-normalised mode (4) gives O = 1
   exactly for V = 1, which the unrounded denominator does not; LSE is the
   unrounded log-sum-exp in every mode;
+* grouped-query attention: scalar loops with the explicit head mapping, and
+  central finite differences for the gradients of a shared K/V head;
 * the near-tie detector (fix_mode 5): counts against scalar loops with
   math.exp and torch's bf16 cast on inputs with near ties but no exact ones,
   and every P_bar below 1 on the rows it raises.
@@ -325,6 +327,53 @@ def emulation_pins(M):
     return failed
 
 
+def gqa_pins(M):
+    """Grouped-query attention: scalar loops with the explicit head mapping
+    (query head h reads key/value head h // group), and the gradient of a
+    shared head against central finite differences of those loops."""
+    failed = []
+    rng = np.random.default_rng(11)
+    B, Hq, Hkv, N, d = 1, 4, 2, 5, 3
+    g = Hq // Hkv
+    q, k, v = _rand(rng, B, Hq, N, d), _rand(rng, B, Hkv, N, d), _rand(rng, B, Hkv, N, d)
+    do = _rand(rng, B, Hq, N, d)
+    sc = 0.7
+
+    def brute_o(qq, kk, vv):
+        out = np.zeros((B, Hq, N, d))
+        for h in range(Hq):
+            hk = h // g
+            for i in range(N):
+                s = [sc * sum(qq[0, h, i, c] * kk[0, hk, j, c] for c in range(d)) for j in range(i + 1)]
+                mx = max(s)
+                e = [math.exp(x - mx) for x in s]
+                tot = sum(e)
+                for c in range(d):
+                    out[0, h, i, c] = sum(e[j] * vv[0, hk, j, c] for j in range(i + 1)) / tot
+        return out
+
+    o, _ = M.attention_fwd(q, M.gqa_expand(k, g), M.gqa_expand(v, g), True, sc)
+    if not np.allclose(o, brute_o(q, k, v), atol=1e-13):
+        failed.append("gqa_forward")
+    _, dk_rep, dv_rep = M.attention_bwd(q, M.gqa_expand(k, g), M.gqa_expand(v, g), do, True, sc)
+    dk, dv = M.gqa_reduce(dk_rep, g), M.gqa_reduce(dv_rep, g)
+    eps = 1e-6
+    for name, arr, grad in (("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            a1, a2 = arr.copy(), arr.copy()
+            a1[idx] += eps
+            a2[idx] -= eps
+            kk1, vv1 = (a1, v) if name == "k" else (k, a1)
+            kk2, vv2 = (a2, v) if name == "k" else (k, a2)
+            num[idx] = (np.sum(do * brute_o(q, kk1, vv1)) - np.sum(do * brute_o(q, kk2, vv2))) / (2 * eps)
+        if not np.allclose(grad, num, rtol=1e-6, atol=1e-8):
+            failed.append(f"gqa_d{name}")
+    if not np.array_equal(M.gqa_reduce(M.gqa_expand(k, g), g), g * np.asarray(k, np.float64)):
+        failed.append("gqa_expand_reduce")
+    return failed
+
+
 # ----------------------------------------------------------------------------
 # the oracle passes every pin
 # ----------------------------------------------------------------------------
@@ -343,6 +392,10 @@ def test_bf16_rounding_matches_torch_cast():
 
 def test_emulation_and_fix_pins():
     assert emulation_pins(ORACLE) == []
+
+
+def test_gqa_pins():
+    assert gqa_pins(ORACLE) == []
 
 
 def test_delta_constant():
@@ -400,6 +453,9 @@ MUTATIONS = [
      "ties = np.sum(raw == raw.max(axis=1, keepdims=True), axis=1, keepdims=True)"),
     ("near_tie_no_shift", "4: 0.0, 5: DELTA_NAT}", "4: 0.0, 5: 0.0}"),
     ("near_tie_threshold_off", "out[b, h] = np.sum(bf16_round(p) == 1.0, axis=1)", "out[b, h] = np.sum(p == 1.0, axis=1)"),
+    ("gqa_expand_wrong_axis", "return np.repeat(_f64(x), group, axis=1)", "return np.tile(_f64(x), (1, group, 1, 1))"),
+    ("gqa_reduce_mean", "return x.reshape(B, H // group, group, N, d).sum(axis=2)",
+     "return x.reshape(B, H // group, group, N, d).mean(axis=2)"),
     ("self_normalised_lse_from_pbar", "lse[b, h] = shift[:, 0] + np.log(l[:, 0])",
      "lse[b, h] = shift[:, 0] + np.log(den[:, 0])"),
 ]
@@ -417,7 +473,7 @@ def _mutant(old, new):
 def test_planted_mistake_is_caught(name, old, new):
     M = _mutant(old, new)
     failed = []
-    for suite in (fwd_pins, bf16_pins, emulation_pins, bwd_pins):
+    for suite in (fwd_pins, bf16_pins, emulation_pins, bwd_pins, gqa_pins):
         try:
             failed += suite(M)
         except Exception as exc:  # a mutant that cannot even run fails its pins
