@@ -158,20 +158,26 @@ bool make_map_dq(CUtensorMap* map, const void* base, int BH, int N, int D) {
 // Shift added to m on repeated-max rows (base-2 units): maps a maximum to 1 - 2^-8.
 const double kDeltaLog2 = -std::log2(1.0 - 1.0 / 256.0);
 
+// H query heads share Hkv key/value heads (H == Hkv: ordinary attention).
+int check_heads(int H, int Hkv) { return (Hkv >= 1 && Hkv <= H && H % Hkv == 0) ? FA_OK : FA_ERR_SHAPE; }
+
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties, int B, int H,
-               int N, int d, int causal, float scale, int fix_mode, cudaStream_t stream) {
+               int Hkv, int N, int d, int causal, float scale, int fix_mode, cudaStream_t stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
   int rc = check_common(B, H, N, d, causal, scale);
   if (rc != FA_OK) return rc;
+  if ((rc = check_heads(H, Hkv)) != FA_OK) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGN;
   if (fix_mode < 0 || fix_mode > 5) return FA_ERR_FIXMODE;
   DeviceState* st = device_state();
   if (!st) return FA_ERR_DEVICE;
   const int BH = B * H;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, BH, N, d) || !make_map(&mk, k, BH, N, d) || !make_map(&mv, v, BH, N, d))
+  if (!make_map(&mq, q, BH, N, d) || !make_map(&mk, k, B * Hkv, N, d) || !make_map(&mv, v, B * Hkv, N, d))
     return FA_ERR_DEVICE;
   FwdParams prm{};
+  prm.H = H;
+  prm.group = H / Hkv;
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.ties = ties;
@@ -213,14 +219,20 @@ extern "C" {
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            int causal, float scale, int fix_mode, void* stream) {
-  return launch_fwd(q, k, v, o, lse, nullptr, B, H, N, d, causal, scale, fix_mode,
+  return launch_fwd(q, k, v, o, lse, nullptr, B, H, H, N, d, causal, scale, fix_mode,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
+               int d, int causal, float scale, int fix_mode, void* stream) {
+  return launch_fwd(q, k, v, o, lse, nullptr, B, H, Hkv, N, d, causal, scale, fix_mode,
                     static_cast<cudaStream_t>(stream));
 }
 
 int fa_fwd_ties(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties, int B, int H,
                 int N, int d, int causal, float scale, int fix_mode, void* stream) {
   if (!ties) return FA_ERR_NULL;
-  return launch_fwd(q, k, v, o, lse, ties, B, H, N, d, causal, scale, fix_mode,
+  return launch_fwd(q, k, v, o, lse, ties, B, H, H, N, d, causal, scale, fix_mode,
                     static_cast<cudaStream_t>(stream));
 }
 
@@ -250,12 +262,19 @@ int fa_bwd_preprocess(const void* o, const void* dout, void* workspace, size_t w
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
-int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dout, void* dk,
-                void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d, int causal,
-                float scale, void* stream) {
+}  // extern "C"
+
+namespace fa {
+namespace {
+
+// The backward main kernel for H query heads sharing Hkv key/value heads.
+int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse, const void* dout, void* dk, void* dv,
+                  void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N, int d, int causal,
+                  float scale, void* stream) {
   if (!q || !k || !v || !lse || !dout || !dk || !dv) return FA_ERR_NULL;
   int rc = check_common(B, H, N, d, causal, scale);
   if (rc != FA_OK) return rc;
+  if ((rc = check_heads(H, Hkv)) != FA_OK) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv))
     return FA_ERR_ALIGN;
   if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, N, d))
@@ -264,8 +283,9 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, c
   if (!st) return FA_ERR_DEVICE;
   const int BH = B * H;
   const size_t rows = size_t(BH) * N;
+  const int BHkv = B * Hkv;
   CUtensorMap mq, mk, mv, mdo, mdq;
-  if (!make_map(&mq, q, BH, N, d) || !make_map(&mk, k, BH, N, d) || !make_map(&mv, v, BH, N, d) ||
+  if (!make_map(&mq, q, BH, N, d) || !make_map(&mk, k, BHkv, N, d) || !make_map(&mv, v, BHkv, N, d) ||
       !make_map(&mdo, dout, BH, N, d) || !make_map_dq(&mdq, workspace, BH, N, d))
     return FA_ERR_DEVICE;
   BwdParams prm{};
@@ -275,13 +295,15 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, c
   prm.dk = static_cast<__nv_bfloat16*>(dk);
   prm.dv = static_cast<__nv_bfloat16*>(dv);
   prm.dev_error = st->dev_error;
-  prm.BH = BH;
+  prm.BH = BHkv;   // work items run over the K/V heads
+  prm.H = H;
+  prm.group = H / Hkv;
   prm.N = N;
   prm.n_kv = (N + 127) / 128;
   prm.causal = causal;
   prm.scale = scale;
   prm.scale_log2 = float(double(scale) * 1.4426950408889634);
-  const int n_items = prm.n_kv * BH;
+  const int n_items = prm.n_kv * BHkv;
   const dim3 grid(unsigned(n_items < st->num_sms ? n_items : st->num_sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const cudaError_t e =
@@ -290,6 +312,17 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, c
                 : launch(fa_bwd_kernel<128>, grid, dim3(BwdLayout<128>::kThreads), BwdLayout<128>::kAlloc, s, mq, mk,
                          mv, mdo, mdq, prm);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dout, void* dk,
+                void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d, int causal,
+                float scale, void* stream) {
+  return bwd_main_impl(q, k, v, lse, dout, dk, dv, workspace, workspace_bytes, B, H, H, N, d, causal, scale, stream);
 }
 
 int fa_bwd_finish(void* dq, const void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale,
@@ -309,13 +342,14 @@ int fa_bwd_finish(void* dq, const void* workspace, size_t workspace_bytes, int B
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
-           void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
-           int causal, float scale, void* stream) {
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+               void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N,
+               int d, int causal, float scale, void* stream) {
   // Check everything up front so that an error leaves every output untouched.
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   int rc = check_common(B, H, N, d, causal, scale);
   if (rc != FA_OK) return rc;
+  if ((rc = check_heads(H, Hkv)) != FA_OK) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv))
     return FA_ERR_ALIGN;
@@ -324,9 +358,16 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if (!device_state()) return FA_ERR_DEVICE;
   rc = fa_bwd_preprocess(o, dout, workspace, workspace_bytes, B, H, N, d, stream);
   if (rc != FA_OK) return rc;
-  rc = fa_bwd_main(q, k, v, lse, dout, dk, dv, workspace, workspace_bytes, B, H, N, d, causal, scale, stream);
+  rc = bwd_main_impl(q, k, v, lse, dout, dk, dv, workspace, workspace_bytes, B, H, Hkv, N, d, causal, scale, stream);
   if (rc != FA_OK) return rc;
   return fa_bwd_finish(dq, workspace, workspace_bytes, B, H, N, d, scale, stream);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+           void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+           int causal, float scale, void* stream) {
+  return fa_bwd_gqa(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, H, N, d, causal, scale,
+                    stream);
 }
 
 const char* fa_status_string(int status) {

@@ -83,7 +83,8 @@ struct BwdParams {
   __nv_bfloat16* dk;    // [BH, N, D]
   __nv_bfloat16* dv;    // [BH, N, D]
   int* dev_error;
-  int BH, N, n_kv, causal;
+  int BH, N, n_kv, causal;   // BH = batch * K/V heads
+  int H, group;         // query heads per batch entry; query heads per K/V head (1 = no sharing)
   float scale, scale_log2;
 };
 
@@ -138,9 +139,12 @@ struct BwdLayout {
 // first (causal: the first key tiles are seen by the most query tiles).  CTAs
 // are persistent and sweep the sorted items with snake_item()
 struct BwdItem {
-  int bh, kv_tile, key0, i_start, n_it;
+  int bh, kv_tile, key0, i_start, n_it_head, n_it;
 };
 
+// One work item = one (batch*K/V head, 128-key tile).  It loops over the
+// query tiles that see those keys, for each query head of the group that
+// shares the K/V head (dK, dV accumulate over all of them): n_it steps.
 __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
   BwdItem w;
   w.kv_tile = item / p.BH;
@@ -148,9 +152,29 @@ __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
   w.key0 = w.kv_tile * 128;
   const int n_q = (p.N + 127) / 128;
   w.i_start = p.causal ? w.kv_tile : 0;
-  w.n_it = n_q - w.i_start;
+  w.n_it_head = n_q - w.i_start;
+  w.n_it = w.n_it_head * p.group;
   return w;
 }
+
+// The steps of an item in order: query tile qt of batch*query-head bh_q,
+// query tiles innermost.  Advanced once per step, without divisions.
+struct BwdSteps {
+  int qt, bh_q, q_first, q_end;
+  __device__ __forceinline__ BwdSteps(const BwdParams& p, const BwdItem& w) {
+    const int hkv = p.H / p.group;
+    q_first = w.i_start;
+    q_end = w.i_start + w.n_it_head;
+    qt = q_first;
+    bh_q = (w.bh / hkv) * p.H + (w.bh % hkv) * p.group;
+  }
+  __device__ __forceinline__ void next() {
+    if (++qt == q_end) {
+      qt = q_first;
+      ++bh_q;
+    }
+  }
+};
 
 // Roles (16 warps):
 //   warps 0-7   key-row math; warp w owns keys 32*(w%4).. (TMEM lane quarter
@@ -274,9 +298,10 @@ __global__ void __launch_bounds__(512, 1)
             tma_load_3d(sk + L::kTileBytes + s * L::kSubBytes, &tm_v, &kv_full[ks], s * 64, w.key0, w.bh, pol_kv);
           }
         }
-        for (int it = 0; it < w.n_it; ++it, ++g) {
+        BwdSteps sp(p, w);
+        for (int it = 0; it < w.n_it; ++it, ++g, sp.next()) {
           const uint32_t st = g % L::kQStages;
-          const int q0 = (w.i_start + it) * 128;
+          const int q0 = sp.qt * 128;
           ok = __all_sync(0xffffffffu, mbar_wait(&q_empty[st], ((g / L::kQStages) & 1) ^ 1, wd));
           if (!ok) break;
           // the Q tile first, so that its load overlaps the LSE/D reads below
@@ -284,7 +309,7 @@ __global__ void __launch_bounds__(512, 1)
             mbar_arrive_expect_tx(&q_full[st], uint32_t(L::kTileBytes));
             for (int s = 0; s < L::kSub; ++s)
               tma_load_3d(smem + L::kQOff + st * L::kTileBytes + s * L::kSubBytes, &tm_q, &q_full[st], s * 64, q0,
-                          w.bh, pol_q);
+                          sp.bh_q, pol_q);
           }
           float* nlse = stats + st * 256;
           float* dd = nlse + 128;
@@ -294,8 +319,8 @@ __global__ void __launch_bounds__(512, 1)
             const int row = q0 + r;
             const bool in = row < p.N;
             // rows past N: P = 2^(-inf) = 0 and D = 0, so they add nothing
-            nlse[r] = in ? -p.lse[size_t(w.bh) * p.N + row] * kLog2e : -__int_as_float(0x7f800000);
-            dd[r] = in ? p.dsum[size_t(w.bh) * p.N + row] : 0.f;
+            nlse[r] = in ? -p.lse[size_t(sp.bh_q) * p.N + row] * kLog2e : -__int_as_float(0x7f800000);
+            dd[r] = in ? p.dsum[size_t(sp.bh_q) * p.N + row] : 0.f;
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&q_full[st]);   // second arrival: the rows are in shared memory
@@ -308,8 +333,9 @@ __global__ void __launch_bounds__(512, 1)
       bool ok = true;
       for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd)) {
         const BwdItem w = bwd_item(p, item);
-        for (int it = 0; it < w.n_it; ++it, ++g) {
-          const int q0 = (w.i_start + it) * 128;
+        BwdSteps sp(p, w);
+        for (int it = 0; it < w.n_it; ++it, ++g, sp.next()) {
+          const int q0 = sp.qt * 128;
           // dO_i: with a single buffer it is refilled once dV_{i-1} has read it
           const uint32_t sd = g % L::kDOStages;
           ok = __all_sync(0xffffffffu, mbar_wait(&do_empty[sd], ((g / L::kDOStages) & 1) ^ 1, wd));
@@ -318,7 +344,7 @@ __global__ void __launch_bounds__(512, 1)
             mbar_arrive_expect_tx(&do_full[sd], uint32_t(L::kTileBytes));
             for (int s = 0; s < L::kSub; ++s)
               tma_load_3d(smem + L::kDOOff + sd * L::kTileBytes + s * L::kSubBytes, &tm_do, &do_full[sd], s * 64,
-                          q0, w.bh, pol_q);
+                          q0, sp.bh_q, pol_q);
           }
           __syncwarp();
         }
@@ -448,9 +474,10 @@ __global__ void __launch_bounds__(512, 1)
     for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd)) {
       const BwdItem w = bwd_item(p, item);
       const bool key_in = w.key0 + kr < p.N;
-      for (int it = 0; it < w.n_it; ++it, ++g) {
+      BwdSteps sp(p, w);
+      for (int it = 0; it < w.n_it; ++it, ++g, sp.next()) {
         const uint32_t st = g % L::kQStages;
-        const int qt = w.i_start + it;
+        const int qt = sp.qt;
         const float* nlse = stats + st * 256 + 64 * half;
         const float* dd = stats + st * 256 + 128 + 64 * half;
         // q_full publishes this stage's LSE/D (written by the producer's lanes)
@@ -574,7 +601,8 @@ __global__ void __launch_bounds__(512, 1)
     bool ok = true;
     for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
       const BwdItem w = bwd_item(p, item);
-      for (int it = 0; it < w.n_it; ++it, ++g) {
+      BwdSteps sp(p, w);
+      for (int it = 0; it < w.n_it; ++it, ++g, sp.next()) {
         ok = __all_sync(0xffffffffu, mbar_wait(dq_full, g & 1, wd));
         if (!ok) break;
         tc_fence_after();
@@ -599,7 +627,7 @@ __global__ void __launch_bounds__(512, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_reduce_add_3d(&tm_dq, box, c * 32, (w.i_start + it) * 128 + wq * 32, w.bh);
+            tma_reduce_add_3d(&tm_dq, box, c * 32, sp.qt * 128 + wq * 32, sp.bh_q);
             bulk_commit();
           }
           ++box_seq;

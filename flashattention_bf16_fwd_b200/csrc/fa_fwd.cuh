@@ -35,7 +35,8 @@ struct FwdParams {
   float* lse;           // [BH, N]
   int32_t* ties;        // [BH, N] or nullptr
   int* dev_error;       // library error flag
-  int BH, N, n_pairs, causal;
+  int BH, N, n_pairs, causal;   // BH = batch * query heads
+  int H, group;         // query heads per batch entry; query heads per K/V head (1 = no sharing)
   float scale_log2;     // scale * log2(e): S -> base-2 exponent domain
   float delta_log2;     // shift added to m on repeated-max rows (0 = fix off)
   float fix_factor;     // 2^-delta_log2: P at a repeated maximum (1 - 2^-8, 0.5 or exp(-1/16))
@@ -170,6 +171,8 @@ __global__ void __launch_bounds__(384, 1)
         bool ok = true;
         for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
           const FwdItem w = fwd_item(p, item);
+          // grouped-query layout: query head h reads K/V head h / group
+          const int kv_bh = (w.bh / p.H) * (p.H / p.group) + (w.bh % p.H) / p.group;
           // the previous item's S MMAs must be done with Q
           if (!(ok = mbar_wait(q_empty, (n_done & 1) ^ 1, wd))) break;
           const int nq = (w.n1 > 0) ? 2 : 1;
@@ -185,8 +188,8 @@ __global__ void __launch_bounds__(384, 1)
             uint8_t* sk = smem + L::kKVOff + st * 2 * L::kTileBytes;
             uint8_t* sv = sk + L::kTileBytes;
             for (int s = 0; s < L::kSub; ++s) {
-              tma_load_3d(sk + s * L::kSubBytes, &tm_k, &kv_full[st], s * 64, j * 128, w.bh, pol_kv);
-              tma_load_3d(sv + s * L::kSubBytes, &tm_v, &kv_full[st], s * 64, j * 128, w.bh, pol_kv);
+              tma_load_3d(sk + s * L::kSubBytes, &tm_k, &kv_full[st], s * 64, j * 128, kv_bh, pol_kv);
+              tma_load_3d(sv + s * L::kSubBytes, &tm_v, &kv_full[st], s * 64, j * 128, kv_bh, pol_kv);
             }
           }
         }

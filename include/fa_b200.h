@@ -113,6 +113,25 @@ FA_API int fa_fwd_ties(const void* q, const void* k, const void* v, void* o, flo
                 float scale, int fix_mode, void* stream);
 
 /*
+ * Grouped-query attention (GQA; MQA when Hkv == 1), the head layout of the
+ * larger Llama 2 models the chibakuma.com page names: H query heads share Hkv
+ * key/value heads, query head h reading key/value head h / (H / Hkv).
+ *   q, o, dout, dq : bf16 [B,H,N,d];  k, v, dk, dv : bf16 [B,Hkv,N,d];
+ *   lse            : float32 [B,H,N].
+ * dK and dV of a shared head are the sums over the query heads of its group.
+ * Hkv must divide H (FA_ERR_SHAPE otherwise).  Everything else is as in
+ * fa_fwd / fa_bwd, which are the Hkv == H case; the workspace is
+ * fa_bwd_workspace_size(B, H, N, d) (query heads).
+ */
+FA_API int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                      int B, int H, int Hkv, int N, int d, int causal, float scale,
+                      int fix_mode, void* stream);
+FA_API int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                      const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                      void* workspace, size_t workspace_bytes, int B, int H, int Hkv,
+                      int N, int d, int causal, float scale, void* stream);
+
+/*
  * fa_bwd_workspace_size - bytes of device scratch fa_bwd needs:
  *   an FP32 dQ accumulator [B,H,N,d] and FP32 D_i = sum_k dO_ik O_ik [B,H,N].
  * Returns 0 for invalid shapes.

@@ -31,7 +31,8 @@ def declared_symbols():
 
 
 def test_header_declares_the_boundary():
-    assert declared_symbols() == sorted(["fa_fwd", "fa_fwd_ties", "fa_bwd_workspace_size", "fa_bwd",
+    assert declared_symbols() == sorted(["fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_bwd_gqa",
+                                         "fa_bwd_workspace_size", "fa_bwd",
                                          "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish",
                                          "fa_bwd_noalloc", "fa_watchdog_selftest", "fa_status_string",
                                          "fa_check_device_error"])
@@ -108,6 +109,24 @@ def test_bwd_argument_errors(fa):
 
 
 FA_ERR_SCRATCH_LIMIT = -11
+
+
+def test_gqa_argument_errors(fa):
+    def fg(H=4, Hkv=2, d=64, q=A):
+        return fa.lib.fa_fwd_gqa(q, A, A, A, A, 1, H, Hkv, 128, d, 1, 0.125, 1, None)
+
+    def bg(H=4, Hkv=2, dk=A):
+        ws = fa.fa_bwd_workspace_size(1, H, 128, 64)
+        return fa.lib.fa_bwd_gqa(A, A, A, A, A, A, A, dk, A, A, ws, 1, H, Hkv, 128, 64, 1, 0.125, None)
+
+    assert fg(Hkv=3) == FA_ERR_SHAPE          # must divide H
+    assert fg(Hkv=0) == FA_ERR_SHAPE
+    assert fg(Hkv=8) == FA_ERR_SHAPE          # more K/V heads than query heads
+    assert fg(d=96) == FA_ERR_HEADDIM
+    assert fg(q=None) == FA_ERR_NULL
+    assert bg(Hkv=3) == FA_ERR_SHAPE
+    assert bg(dk=MIS) == FA_ERR_ALIGN
+    assert bg(dk=None) == FA_ERR_NULL
 
 
 def test_bwd_noalloc_argument_errors(fa):
