@@ -35,6 +35,10 @@ What it computes, and where each step is stated:
   keeps the plain shift but divides by the sum of the rounded P_bar instead of
   the unrounded P (a self-normalised output).  LSE is the unrounded
   log-sum-exp in every mode.
+* The same in FP16 (the pages treat FP16 and BF16 together as the
+  low-precision formats of the instability: yicaiai article, abstract):
+  P_bar rounded to fp16, and the fix maps the maxima to 1 - 2^-11, the
+  largest fp16 value below 1.
 * Grouped-query attention (GQA/MQA head layouts, the Llama 2 family the
   chibakuma.com page names): H_q query heads share H_kv key/value heads,
   query head h reading key/value head h // (H_q / H_kv).  The forward is the
@@ -53,7 +57,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "DELTA_LOG2", "DELTA_NAT", "FIX_SHIFT_NAT", "SELF_NORMALISED_MODES", "NEAR_TIE_MODES", "bf16_round", "scores", "attention_fwd",
+    "DELTA_LOG2", "DELTA_NAT", "DELTA16_NAT", "fp16_round", "FIX_SHIFT_NAT", "SELF_NORMALISED_MODES", "NEAR_TIE_MODES", "bf16_round", "scores", "attention_fwd",
     "attention_bwd", "attention_fwd_bf16p", "tie_counts", "near_tie_counts", "gqa_expand", "gqa_reduce",
 ]
 
@@ -68,6 +72,10 @@ NEAR_TIE_MODES = (5,)
 SELF_NORMALISED_MODES = (4,)
 
 _BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
+_FP16_MAX = (2.0 - 2.0 ** -10) * 2.0 ** 15
+
+# The fix's shift for fp16 P_bar (natural-log units): maxima -> 1 - 2^-11.
+DELTA16_NAT = -np.log(1.0 - 2.0 ** -11)
 
 
 def bf16_round(x) -> np.ndarray:
@@ -87,6 +95,27 @@ def bf16_round(x) -> np.ndarray:
     r = np.ldexp(np.rint(np.ldexp(xf, -q_exp)), q_exp)
     r = np.where(np.abs(r) > _BF16_MAX, np.copysign(np.inf, xf), r)
     # keep the sign of values that round to zero
+    r = np.where(r == 0.0, np.copysign(0.0, xf), r)
+    out[fin] = r
+    return out
+
+
+def fp16_round(x) -> np.ndarray:
+    """Round to the nearest IEEE binary16 value, ties to even, returned as float64.
+
+    fp16 keeps 11 significant bits: the quantum of a normal value in
+    [2^(e-1), 2^e) is 2^(e-11); below 2^-14 the quantum is fixed at 2^-24
+    (subnormals).  Results beyond 65504 become infinities; NaN stays NaN; the
+    sign of zero is kept.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = x.copy()
+    fin = np.isfinite(x) & (x != 0.0)
+    xf = x[fin]
+    _, e = np.frexp(xf)
+    q_exp = np.maximum(e, -13) - 11
+    r = np.ldexp(np.rint(np.ldexp(xf, -q_exp)), q_exp)
+    r = np.where(np.abs(r) > _FP16_MAX, np.copysign(np.inf, xf), r)
     r = np.where(r == 0.0, np.copysign(0.0, xf), r)
     out[fin] = r
     return out
@@ -197,7 +226,7 @@ def near_tie_counts(q, k, causal: bool, scale: float) -> np.ndarray:
 
 
 def attention_fwd_bf16p(q, k, v, causal: bool, scale: float, fix_mode: int,
-                        round_p: bool = True, return_pbar: bool = False):
+                        round_p: bool = True, return_pbar: bool = False, fmt: str = "bf16"):
     """Attention with the safe-softmax shift, BF16-rounded P_bar and the fix.
 
     Per row i (one shift for the whole row):
@@ -213,9 +242,15 @@ def attention_fwd_bf16p(q, k, v, causal: bool, scale: float, fix_mode: int,
     P_bar == 1 exactly; fix_mode 1 maps them to 1 - 2^-8, fix_mode 2 to 0.5,
     fix_mode 3 to exp(-1/16); fix_mode 4 keeps them at 1 and self-normalises;
     fix_mode 5 is fix_mode 1 triggered by near ties.
+    fmt = "fp16" rounds P_bar to fp16 instead (fix_mode 0 or 1 only; the fix
+    then maps the maxima to 1 - 2^-11).
     """
     if fix_mode not in FIX_SHIFT_NAT:
         raise ValueError("fix_mode must be 0, 1, 2, 3, 4 or 5")
+    if fmt not in ("bf16", "fp16") or (fmt == "fp16" and fix_mode not in (0, 1)):
+        raise ValueError("fmt must be bf16, or fp16 with fix_mode 0 or 1")
+    round_fn = bf16_round if fmt == "bf16" else fp16_round
+    shifts = FIX_SHIFT_NAT if fmt == "bf16" else {0: 0.0, 1: DELTA16_NAT}
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, N, d = q.shape
     o = np.empty((B, H, N, v.shape[-1]))
@@ -227,13 +262,13 @@ def attention_fwd_bf16p(q, k, v, causal: bool, scale: float, fix_mode: int,
         s = scale * raw
         m = s.max(axis=1, keepdims=True)
         if fix_mode in NEAR_TIE_MODES:
-            ties = np.sum(bf16_round(np.exp(s - m)) == 1.0, axis=1, keepdims=True)
+            ties = np.sum(round_fn(np.exp(s - m)) == 1.0, axis=1, keepdims=True)
         else:
             ties = np.sum(raw == raw.max(axis=1, keepdims=True), axis=1, keepdims=True)
-        shift = m + FIX_SHIFT_NAT[fix_mode] * (ties >= 2)
+        shift = m + shifts[fix_mode] * (ties >= 2)
         p = np.exp(s - shift)
         l = p.sum(axis=1, keepdims=True)
-        pbar = bf16_round(p) if round_p else p
+        pbar = round_fn(p) if round_p else p
         den = pbar.sum(axis=1, keepdims=True) if fix_mode in SELF_NORMALISED_MODES else l
         o[b, h] = (pbar @ v[b, h]) / den
         lse[b, h] = shift[:, 0] + np.log(l[:, 0])

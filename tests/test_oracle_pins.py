@@ -19,6 +19,8 @@ The pages print no worked example, so the oracle is pinned by
   unrounded log-sum-exp in every mode;
 * grouped-query attention: scalar loops with the explicit head mapping, and
   central finite differences for the gradients of a shared K/V head;
+* fp16 rounding against torch's fp16 cast, and the fix with fp16 P_bar
+  (maxima at 1 - 2^-11);
 * the near-tie detector (fix_mode 5): counts against scalar loops with
   math.exp and torch's bf16 cast on inputs with near ties but no exact ones,
   and every P_bar below 1 on the rows it raises.
@@ -193,6 +195,44 @@ def bf16_pins(M):
     nan = M.bf16_round(np.array([np.nan]))
     if not np.isnan(nan).all():
         failed.append("nan")
+    return failed
+
+
+def fp16_pins(M):
+    """fp16 rounding against torch's float32 -> float16 cast, and the fix's
+    property with fp16 P_bar: the maxima of repeated-max rows land on
+    1 - 2^-11, the largest fp16 value below 1."""
+    failed = []
+    rng = np.random.default_rng(13)
+    x = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32),
+        (rng.standard_normal(20000) * 1e-6).astype(np.float32),     # fp16 subnormals
+        (rng.standard_normal(5000) * 3e4).astype(np.float32),
+        np.exp(rng.uniform(-20, 0, 20000)).astype(np.float32),
+    ])
+    edges = np.array([0.0, -0.0, 1.0, 1 - 2 ** -12, 1 - 3 * 2 ** -12, 1 - 2 ** -11, 2.0 ** -14, 2.0 ** -24,
+                      2.0 ** -25, 3 * 2.0 ** -26, 65504.0, 65519.0, 65520.0, 7e4, np.inf], dtype=np.float32)
+    x = np.concatenate([x, edges, -edges])
+    ref = torch.from_numpy(x).to(torch.float16).to(torch.float64).numpy()
+    got = M.fp16_round(x.astype(np.float64))
+    if not (np.all((got == ref) | (np.isnan(got) & np.isnan(ref))) and np.all(np.signbit(got) == np.signbit(ref))):
+        failed.append("fp16_torch_cast")
+    q, k, v = _tie_inputs(rng)
+    ties = np.stack([np.asarray(brute_ties(q[0, h].tolist(), k[0, h].tolist(), True)) for h in range(2)])
+    _, _, p1 = M.attention_fwd_bf16p(q, k, v, True, 0.5, 1, return_pbar=True, fmt="fp16")
+    _, _, p0 = M.attention_fwd_bf16p(q, k, v, True, 0.5, 0, return_pbar=True, fmt="fp16")
+    ok = True
+    for h in range(2):
+        for i in range(q.shape[2]):
+            r1, r0 = p1[0, h, i, : i + 1], p0[0, h, i, : i + 1]
+            if ties[h, i] >= 2:
+                ok &= r1.max() == 1.0 - 2.0 ** -11 and np.sum(r1 == 1.0 - 2.0 ** -11) == ties[h, i]
+            else:
+                ok &= np.array_equal(r1, r0) and r0.max() == 1.0
+            # P_bar is on the fp16 grid (torch's cast, not the oracle's)
+            ok &= np.array_equal(torch.from_numpy(r1).to(torch.float16).double().numpy(), r1)
+    if not ok:
+        failed.append("fp16_fix_property")
     return failed
 
 
@@ -398,6 +438,10 @@ def test_gqa_pins():
     assert gqa_pins(ORACLE) == []
 
 
+def test_fp16_pins():
+    assert fp16_pins(ORACLE) == []
+
+
 def test_delta_constant():
     # the shift maps a maximum to exactly the largest bf16 value below 1
     assert ORACLE.bf16_round(np.exp(-ORACLE.DELTA_NAT)) == 0.99609375
@@ -440,22 +484,27 @@ MUTATIONS = [
     ("dk_not_transposed", "dk[b, h] = scale * (ds.T @ q[b, h])", "dk[b, h] = scale * (ds @ q[b, h])"),
     ("dq_drops_scale", "dq[b, h] = scale * (ds @ k[b, h])", "dq[b, h] = (ds @ k[b, h])"),
     ("bf16_one_bit_short", "q_exp = np.maximum(e, -125) - 8", "q_exp = np.maximum(e, -125) - 7"),
-    ("bf16_truncates", "np.rint(np.ldexp(xf, -q_exp))", "np.trunc(np.ldexp(xf, -q_exp))"),
+    ("bf16_truncates", "q_exp = np.maximum(e, -125) - 8\n    r = np.ldexp(np.rint(np.ldexp(xf, -q_exp)), q_exp)",
+     "q_exp = np.maximum(e, -125) - 8\n    r = np.ldexp(np.trunc(np.ldexp(xf, -q_exp)), q_exp)"),
     ("bf16_no_subnormals", "q_exp = np.maximum(e, -125) - 8", "q_exp = e - 8"),
     ("fix_on_every_row", "* (ties >= 2)", "* (ties >= 1)"),
     ("fix_wrong_delta", "DELTA_NAT = -np.log(1.0 - 2.0 ** -8)", "DELTA_NAT = -np.log(1.0 - 2.0 ** -6)"),
-    ("emulation_skips_rounding", "pbar = bf16_round(p) if round_p else p", "pbar = p"),
+    ("emulation_skips_rounding", "pbar = round_fn(p) if round_p else p", "pbar = p"),
     ("ties_ignore_mask", "s = np.where(vis, q[b, h] @ k[b, h].T, -np.inf)\n        out[b, h]", "s = q[b, h] @ k[b, h].T\n        out[b, h]"),
     ("variant_shift_in_log2", "2: float(np.log(2.0))", "2: 1.0"),
     ("variant_off_grid_value", "3: 1.0 / 16.0", "3: 1.0 / 8.0"),
     ("self_normalised_unrounded_den", "den = pbar.sum(axis=1, keepdims=True) if", "den = l if"),
-    ("near_ties_count_exact_ties", "ties = np.sum(bf16_round(np.exp(s - m)) == 1.0, axis=1, keepdims=True)",
+    ("near_ties_count_exact_ties", "ties = np.sum(round_fn(np.exp(s - m)) == 1.0, axis=1, keepdims=True)",
      "ties = np.sum(raw == raw.max(axis=1, keepdims=True), axis=1, keepdims=True)"),
     ("near_tie_no_shift", "4: 0.0, 5: DELTA_NAT}", "4: 0.0, 5: 0.0}"),
     ("near_tie_threshold_off", "out[b, h] = np.sum(bf16_round(p) == 1.0, axis=1)", "out[b, h] = np.sum(p == 1.0, axis=1)"),
     ("gqa_expand_wrong_axis", "return np.repeat(_f64(x), group, axis=1)", "return np.tile(_f64(x), (1, group, 1, 1))"),
     ("gqa_reduce_mean", "return x.reshape(B, H // group, group, N, d).sum(axis=2)",
      "return x.reshape(B, H // group, group, N, d).mean(axis=2)"),
+    ("fp16_one_bit_short", "q_exp = np.maximum(e, -13) - 11", "q_exp = np.maximum(e, -13) - 10"),
+    ("fp16_no_subnormals", "q_exp = np.maximum(e, -13) - 11", "q_exp = e - 11"),
+    ("fp16_fix_bf16_delta", "shifts = FIX_SHIFT_NAT if fmt == \"bf16\" else {0: 0.0, 1: DELTA16_NAT}",
+     "shifts = FIX_SHIFT_NAT"),
     ("self_normalised_lse_from_pbar", "lse[b, h] = shift[:, 0] + np.log(l[:, 0])",
      "lse[b, h] = shift[:, 0] + np.log(den[:, 0])"),
 ]
@@ -473,7 +522,7 @@ def _mutant(old, new):
 def test_planted_mistake_is_caught(name, old, new):
     M = _mutant(old, new)
     failed = []
-    for suite in (fwd_pins, bf16_pins, emulation_pins, bwd_pins, gqa_pins):
+    for suite in (fwd_pins, bf16_pins, emulation_pins, bwd_pins, gqa_pins, fp16_pins):
         try:
             failed += suite(M)
         except Exception as exc:  # a mutant that cannot even run fails its pins
