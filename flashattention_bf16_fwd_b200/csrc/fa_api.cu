@@ -61,33 +61,24 @@ DeviceState* device_state() {
     if (cudaGetSymbolAddress(&addr, g_dev_error) != cudaSuccess) return;
     st->dev_error = static_cast<int*>(addr);
     bool ok = true;
-    ok &= cudaFuncSetAttribute(fa_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               FwdLayout<64>::kAlloc) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(fa_fwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               FwdLayout<128>::kAlloc) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(fa_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               FwdLayout<64>::kAlloc) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(fa_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               FwdLayout<128>::kAlloc) == cudaSuccess;
-    // The forward kernel moves registers between warpgroups with setmaxnreg;
-    // the split assumes exactly kLaunchRegs registers per thread at launch.
-    cudaFuncAttributes fattr{};
-    ok &= cudaFuncGetAttributes(&fattr, fa_fwd_kernel<64, false>) == cudaSuccess &&
-          fattr.numRegs == FwdLayout<64>::kLaunchRegs;
-    ok &= cudaFuncGetAttributes(&fattr, fa_fwd_kernel<128, false>) == cudaSuccess &&
-          fattr.numRegs == FwdLayout<128>::kLaunchRegs;
-    ok &= cudaFuncGetAttributes(&fattr, fa_fwd_kernel<64, true>) == cudaSuccess &&
-          fattr.numRegs == FwdLayout<64>::kLaunchRegs;
-    ok &= cudaFuncGetAttributes(&fattr, fa_fwd_kernel<128, true>) == cudaSuccess &&
-          fattr.numRegs == FwdLayout<128>::kLaunchRegs;
-    ok &= cudaFuncGetAttributes(&fattr, fa_bwd_kernel<64>) == cudaSuccess &&
-          fattr.numRegs == BwdLayout<64>::kLaunchRegs;
-    ok &= cudaFuncGetAttributes(&fattr, fa_bwd_kernel<128>) == cudaSuccess &&
-          fattr.numRegs == BwdLayout<128>::kLaunchRegs;
-    ok &= cudaFuncSetAttribute(fa_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               BwdLayout<64>::kAlloc) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(fa_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               BwdLayout<128>::kAlloc) == cudaSuccess;
+    // Every kernel instantiation: large shared memory, and the register count
+    // at launch that its setmaxnreg split assumes (a miscounted pool would stall
+    // setmaxnreg.inc).
+    auto setup = [&](auto kernel, int smem, int regs) {
+      cudaFuncAttributes fattr{};
+      ok &= cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+      ok &= cudaFuncGetAttributes(&fattr, kernel) == cudaSuccess && fattr.numRegs == regs;
+    };
+    setup(fa_fwd_kernel<64, false, ElemBF16>, FwdLayout<64>::kAlloc, FwdLayout<64>::kLaunchRegs);
+    setup(fa_fwd_kernel<128, false, ElemBF16>, FwdLayout<128>::kAlloc, FwdLayout<128>::kLaunchRegs);
+    setup(fa_fwd_kernel<64, true, ElemBF16>, FwdLayout<64>::kAlloc, FwdLayout<64>::kLaunchRegs);
+    setup(fa_fwd_kernel<128, true, ElemBF16>, FwdLayout<128>::kAlloc, FwdLayout<128>::kLaunchRegs);
+    setup(fa_fwd_kernel<64, false, ElemF16>, FwdLayout<64>::kAlloc, FwdLayout<64>::kLaunchRegs);
+    setup(fa_fwd_kernel<128, false, ElemF16>, FwdLayout<128>::kAlloc, FwdLayout<128>::kLaunchRegs);
+    setup(fa_bwd_kernel<64, ElemBF16>, BwdLayout<64>::kAlloc, BwdLayout<64>::kLaunchRegs);
+    setup(fa_bwd_kernel<128, ElemBF16>, BwdLayout<128>::kAlloc, BwdLayout<128>::kLaunchRegs);
+    setup(fa_bwd_kernel<64, ElemF16>, BwdLayout<64>::kAlloc, BwdLayout<64>::kLaunchRegs);
+    setup(fa_bwd_kernel<128, ElemF16>, BwdLayout<128>::kAlloc, BwdLayout<128>::kLaunchRegs);
     st->ok = ok ? 1 : 0;
   });
   return st->ok ? st : nullptr;
@@ -129,14 +120,15 @@ int check_common(int B, int H, int N, int d, int causal, float scale) {
 
 // A [BH, N, D] bf16 tensor seen as 3-D (d, n, bh); boxes of 64 x 128 x 1 with
 // the 128-byte swizzle the tcgen05 descriptors expect.  Rows past N read 0.
-bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D,
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(N), cuuint64_t(BH)};
   cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(N) * D * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  return enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -157,23 +149,34 @@ bool make_map_dq(CUtensorMap* map, const void* base, int BH, int N, int D) {
 
 // Shift added to m on repeated-max rows (base-2 units): maps a maximum to 1 - 2^-8.
 const double kDeltaLog2 = -std::log2(1.0 - 1.0 / 256.0);
+// The same for fp16 P_bar: maps a maximum to 1 - 2^-11.
+const double kDeltaLog2F16 = -std::log2(1.0 - 1.0 / 2048.0);
+
+template <typename E>
+constexpr CUtensorMapDataType map_type() {
+  return E::kMmaFmt == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+}
 
 // H query heads share Hkv key/value heads (H == Hkv: ordinary attention).
 int check_heads(int H, int Hkv) { return (Hkv >= 1 && Hkv <= H && H % Hkv == 0) ? FA_OK : FA_ERR_SHAPE; }
 
+template <typename E>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties, int B, int H,
                int Hkv, int N, int d, int causal, float scale, int fix_mode, cudaStream_t stream) {
+  constexpr bool kF16 = E::kMmaFmt == 0;
   if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
   int rc = check_common(B, H, N, d, causal, scale);
   if (rc != FA_OK) return rc;
   if ((rc = check_heads(H, Hkv)) != FA_OK) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGN;
-  if (fix_mode < 0 || fix_mode > 5) return FA_ERR_FIXMODE;
+  if (fix_mode < 0 || fix_mode > (kF16 ? 1 : 5)) return FA_ERR_FIXMODE;
   DeviceState* st = device_state();
   if (!st) return FA_ERR_DEVICE;
   const int BH = B * H;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, BH, N, d) || !make_map(&mk, k, B * Hkv, N, d) || !make_map(&mv, v, B * Hkv, N, d))
+  constexpr CUtensorMapDataType dt = map_type<E>();
+  if (!make_map(&mq, q, BH, N, d, dt) || !make_map(&mk, k, B * Hkv, N, d, dt) ||
+      !make_map(&mv, v, B * Hkv, N, d, dt))
     return FA_ERR_DEVICE;
   FwdParams prm{};
   prm.H = H;
@@ -189,7 +192,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   prm.scale_log2 = float(double(scale) * 1.4426950408889634);
   // shift on repeated-max rows per fix_mode, in base-2 units: 1 and 5 map the
   // maxima to 1 - 2^-8, 2 to 0.5, 3 to exp(-1/16); 0 and 4 keep the plain shift
-  const double delta = (fix_mode == 1 || fix_mode == 5) ? kDeltaLog2
+  const double delta = (fix_mode == 1 && kF16)           ? kDeltaLog2F16
+                       : (fix_mode == 1 || fix_mode == 5) ? kDeltaLog2
                        : fix_mode == 2                  ? 1.0
                        : fix_mode == 3                  ? 1.4426950408889634 / 16.0
                                                         : 0.0;
@@ -201,8 +205,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   const int n_items = prm.n_pairs * BH;
   const dim3 grid(unsigned(n_items < st->num_sms ? n_items : st->num_sms));
   const bool variants = fix_mode >= 4;   // self-normalised or near-tie code
-  auto kern = (d == 64) ? (variants ? fa_fwd_kernel<64, true> : fa_fwd_kernel<64, false>)
-                        : (variants ? fa_fwd_kernel<128, true> : fa_fwd_kernel<128, false>);
+  auto kern = (d == 64) ? (variants ? fa_fwd_kernel<64, !kF16, E> : fa_fwd_kernel<64, false, E>)
+                        : (variants ? fa_fwd_kernel<128, !kF16, E> : fa_fwd_kernel<128, false, E>);
   const int smem = (d == 64) ? FwdLayout<64>::kAlloc : FwdLayout<128>::kAlloc;
   const cudaError_t e = launch(kern, grid, dim3(FwdLayout<64>::kThreads), smem, stream, mq, mk, mv, prm);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
@@ -219,20 +223,26 @@ extern "C" {
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            int causal, float scale, int fix_mode, void* stream) {
-  return launch_fwd(q, k, v, o, lse, nullptr, B, H, H, N, d, causal, scale, fix_mode,
-                    static_cast<cudaStream_t>(stream));
+  return launch_fwd<ElemBF16>(q, k, v, o, lse, nullptr, B, H, H, N, d, causal, scale, fix_mode,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+               int causal, float scale, int fix_mode, void* stream) {
+  return launch_fwd<ElemF16>(q, k, v, o, lse, nullptr, B, H, H, N, d, causal, scale, fix_mode,
+                             static_cast<cudaStream_t>(stream));
 }
 
 int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
                int d, int causal, float scale, int fix_mode, void* stream) {
-  return launch_fwd(q, k, v, o, lse, nullptr, B, H, Hkv, N, d, causal, scale, fix_mode,
+  return launch_fwd<ElemBF16>(q, k, v, o, lse, nullptr, B, H, Hkv, N, d, causal, scale, fix_mode,
                     static_cast<cudaStream_t>(stream));
 }
 
 int fa_fwd_ties(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties, int B, int H,
                 int N, int d, int causal, float scale, int fix_mode, void* stream) {
   if (!ties) return FA_ERR_NULL;
-  return launch_fwd(q, k, v, o, lse, ties, B, H, H, N, d, causal, scale, fix_mode,
+  return launch_fwd<ElemBF16>(q, k, v, o, lse, ties, B, H, H, N, d, causal, scale, fix_mode,
                     static_cast<cudaStream_t>(stream));
 }
 
@@ -242,8 +252,15 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
 }
 
-int fa_bwd_preprocess(const void* o, const void* dout, void* workspace, size_t workspace_bytes, int B, int H,
-                      int N, int d, void* stream) {
+}  // extern "C"
+
+namespace fa {
+namespace {
+
+// The backward's three launches for element format E.
+template <typename E>
+int pre_impl(const void* o, const void* dout, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+             void* stream) {
   if (!o || !dout) return FA_ERR_NULL;
   int rc = check_common(B, H, N, d, 0, 1.f);
   if (rc != FA_OK) return rc;
@@ -256,18 +273,15 @@ int fa_bwd_preprocess(const void* o, const void* dout, void* workspace, size_t w
   float* dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256(rows * d * sizeof(float)));
   const int threads = 256;
   const long long blocks = ((long long)rows * 8 + threads - 1) / threads;
-  const cudaError_t e = launch(fa_bwd_pre_kernel, dim3(unsigned(blocks)), dim3(threads), 0,
-                               static_cast<cudaStream_t>(stream), static_cast<const __nv_bfloat16*>(o),
-                               static_cast<const __nv_bfloat16*>(dout), dsum, dq_acc, (long long)rows, d);
+  using T = typename E::T;
+  const cudaError_t e = launch(fa_bwd_pre_kernel<E>, dim3(unsigned(blocks)), dim3(threads), 0,
+                               static_cast<cudaStream_t>(stream), static_cast<const T*>(o),
+                               static_cast<const T*>(dout), dsum, dq_acc, (long long)rows, d);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
-}  // extern "C"
-
-namespace fa {
-namespace {
-
 // The backward main kernel for H query heads sharing Hkv key/value heads.
+template <typename E>
 int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse, const void* dout, void* dk, void* dv,
                   void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N, int d, int causal,
                   float scale, void* stream) {
@@ -284,16 +298,17 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse,
   const int BH = B * H;
   const size_t rows = size_t(BH) * N;
   const int BHkv = B * Hkv;
+  constexpr CUtensorMapDataType dt = map_type<E>();
   CUtensorMap mq, mk, mv, mdo, mdq;
-  if (!make_map(&mq, q, BH, N, d) || !make_map(&mk, k, BHkv, N, d) || !make_map(&mv, v, BHkv, N, d) ||
-      !make_map(&mdo, dout, BH, N, d) || !make_map_dq(&mdq, workspace, BH, N, d))
+  if (!make_map(&mq, q, BH, N, d, dt) || !make_map(&mk, k, BHkv, N, d, dt) || !make_map(&mv, v, BHkv, N, d, dt) ||
+      !make_map(&mdo, dout, BH, N, d, dt) || !make_map_dq(&mdq, workspace, BH, N, d))
     return FA_ERR_DEVICE;
   BwdParams prm{};
   prm.lse = lse;
   prm.dsum = reinterpret_cast<const float*>(static_cast<uint8_t*>(workspace) + align256(rows * d * sizeof(float)));
   prm.dq_acc = static_cast<float*>(workspace);
-  prm.dk = static_cast<__nv_bfloat16*>(dk);
-  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.dk = dk;
+  prm.dv = dv;
   prm.dev_error = st->dev_error;
   prm.BH = BHkv;   // work items run over the K/V heads
   prm.H = H;
@@ -307,26 +322,16 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse,
   const dim3 grid(unsigned(n_items < st->num_sms ? n_items : st->num_sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const cudaError_t e =
-      (d == 64) ? launch(fa_bwd_kernel<64>, grid, dim3(BwdLayout<64>::kThreads), BwdLayout<64>::kAlloc, s, mq, mk, mv,
-                         mdo, mdq, prm)
-                : launch(fa_bwd_kernel<128>, grid, dim3(BwdLayout<128>::kThreads), BwdLayout<128>::kAlloc, s, mq, mk,
-                         mv, mdo, mdq, prm);
+      (d == 64) ? launch(fa_bwd_kernel<64, E>, grid, dim3(BwdLayout<64>::kThreads), BwdLayout<64>::kAlloc, s, mq, mk,
+                         mv, mdo, mdq, prm)
+                : launch(fa_bwd_kernel<128, E>, grid, dim3(BwdLayout<128>::kThreads), BwdLayout<128>::kAlloc, s, mq,
+                         mk, mv, mdo, mdq, prm);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
-}  // namespace
-}  // namespace fa
-
-extern "C" {
-
-int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dout, void* dk,
-                void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d, int causal,
-                float scale, void* stream) {
-  return bwd_main_impl(q, k, v, lse, dout, dk, dv, workspace, workspace_bytes, B, H, H, N, d, causal, scale, stream);
-}
-
-int fa_bwd_finish(void* dq, const void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale,
-                  void* stream) {
+template <typename E>
+int finish_impl(void* dq, const void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale,
+                void* stream) {
   if (!dq) return FA_ERR_NULL;
   int rc = check_common(B, H, N, d, 0, scale);
   if (rc != FA_OK) return rc;
@@ -336,15 +341,16 @@ int fa_bwd_finish(void* dq, const void* workspace, size_t workspace_bytes, int B
   if (!device_state()) return FA_ERR_DEVICE;
   const long long n8 = (long long)B * H * N * d / 8;
   const int threads = 256;
-  const cudaError_t e = launch(fa_bwd_dq_kernel, dim3(unsigned((n8 + threads - 1) / threads)), dim3(threads), 0,
+  const cudaError_t e = launch(fa_bwd_dq_kernel<E>, dim3(unsigned((n8 + threads - 1) / threads)), dim3(threads), 0,
                                static_cast<cudaStream_t>(stream), static_cast<const float*>(workspace),
-                               static_cast<__nv_bfloat16*>(dq), scale, n8);
+                               static_cast<typename E::T*>(dq), scale, n8);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
-int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
-               void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N,
-               int d, int causal, float scale, void* stream) {
+template <typename E>
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
+             void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N, int d,
+             int causal, float scale, void* stream) {
   // Check everything up front so that an error leaves every output untouched.
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   int rc = check_common(B, H, N, d, causal, scale);
@@ -356,18 +362,55 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
   if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, N, d))
     return FA_ERR_WORKSPACE;
   if (!device_state()) return FA_ERR_DEVICE;
-  rc = fa_bwd_preprocess(o, dout, workspace, workspace_bytes, B, H, N, d, stream);
+  rc = pre_impl<E>(o, dout, workspace, workspace_bytes, B, H, N, d, stream);
   if (rc != FA_OK) return rc;
-  rc = bwd_main_impl(q, k, v, lse, dout, dk, dv, workspace, workspace_bytes, B, H, Hkv, N, d, causal, scale, stream);
+  rc = bwd_main_impl<E>(q, k, v, lse, dout, dk, dv, workspace, workspace_bytes, B, H, Hkv, N, d, causal, scale,
+                        stream);
   if (rc != FA_OK) return rc;
-  return fa_bwd_finish(dq, workspace, workspace_bytes, B, H, N, d, scale, stream);
+  return finish_impl<E>(dq, workspace, workspace_bytes, B, H, N, d, scale, stream);
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+int fa_bwd_preprocess(const void* o, const void* dout, void* workspace, size_t workspace_bytes, int B, int H,
+                      int N, int d, void* stream) {
+  return pre_impl<ElemBF16>(o, dout, workspace, workspace_bytes, B, H, N, d, stream);
+}
+
+int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dout, void* dk,
+                void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d, int causal,
+                float scale, void* stream) {
+  return bwd_main_impl<ElemBF16>(q, k, v, lse, dout, dk, dv, workspace, workspace_bytes, B, H, H, N, d, causal,
+                                 scale, stream);
+}
+
+int fa_bwd_finish(void* dq, const void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale,
+                  void* stream) {
+  return finish_impl<ElemBF16>(dq, workspace, workspace_bytes, B, H, N, d, scale, stream);
+}
+
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+               void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N,
+               int d, int causal, float scale, void* stream) {
+  return bwd_impl<ElemBF16>(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, N, d, causal,
+                            scale, stream);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
            void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
            int causal, float scale, void* stream) {
-  return fa_bwd_gqa(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, H, N, d, causal, scale,
-                    stream);
+  return bwd_impl<ElemBF16>(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, H, N, d, causal,
+                            scale, stream);
+}
+
+int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+               void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+               int causal, float scale, void* stream) {
+  return bwd_impl<ElemF16>(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, H, N, d, causal,
+                           scale, stream);
 }
 
 const char* fa_status_string(int status) {

@@ -22,8 +22,9 @@ namespace fa {
 
 // D_i = sum_k dO_ik O_ik in FP32; also zeroes the FP32 dQ accumulator.
 // Eight threads per row; each covers d/8 consecutive elements.
-__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
-                                                         const __nv_bfloat16* __restrict__ dout,
+template <typename E>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const typename E::T* __restrict__ o,
+                                                         const typename E::T* __restrict__ dout,
                                                          float* __restrict__ dsum, float* __restrict__ dq_acc,
                                                          long long rows, int d) {
   grid_dep_wait();
@@ -38,12 +39,12 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
     for (int c = 0; c < per; c += 8) {
       const uint4 a = *reinterpret_cast<const uint4*>(o + base + c);
       const uint4 b = *reinterpret_cast<const uint4*>(dout + base + c);
-      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+      const uint32_t* a2 = reinterpret_cast<const uint32_t*>(&a);
+      const uint32_t* b2 = reinterpret_cast<const uint32_t*>(&b);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float2 fa = __bfloat1622float2(a2[i]);
-        const float2 fb = __bfloat1622float2(b2[i]);
+        const float2 fa = E::unpack(a2[i]);
+        const float2 fb = E::unpack(b2[i]);
         acc = fmaf(fa.x, fb.x, acc);
         acc = fmaf(fa.y, fb.y, acc);
       }
@@ -59,8 +60,9 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
 }
 
 // dQ = scale * accumulator, eight elements per thread.
+template <typename E>
 __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict__ acc,
-                                                        __nv_bfloat16* __restrict__ dq, float scale,
+                                                        typename E::T* __restrict__ dq, float scale,
                                                         long long n8) {
   grid_dep_wait();
   grid_dep_launch();
@@ -69,10 +71,10 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict_
   const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
   const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
   uint4 w;
-  w.x = pack_bf16(a.x * scale, a.y * scale);
-  w.y = pack_bf16(a.z * scale, a.w * scale);
-  w.z = pack_bf16(b.x * scale, b.y * scale);
-  w.w = pack_bf16(b.z * scale, b.w * scale);
+  w.x = E::pack(a.x * scale, a.y * scale);
+  w.y = E::pack(a.z * scale, a.w * scale);
+  w.z = E::pack(b.x * scale, b.y * scale);
+  w.w = E::pack(b.z * scale, b.w * scale);
   reinterpret_cast<uint4*>(dq)[i] = w;
 }
 
@@ -80,8 +82,8 @@ struct BwdParams {
   const float* lse;     // [BH, N] natural log
   const float* dsum;    // [BH, N] D_i
   float* dq_acc;        // [BH, N, D] FP32
-  __nv_bfloat16* dk;    // [BH, N, D]
-  __nv_bfloat16* dv;    // [BH, N, D]
+  void* dk;             // [BH, N, D] of the element type
+  void* dv;             // [BH, N, D] of the element type
   int* dev_error;
   int BH, N, n_kv, causal;   // BH = batch * K/V heads
   int H, group;         // query heads per batch entry; query heads per K/V head (1 = no sharing)
@@ -191,7 +193,9 @@ struct BwdSteps {
 //   dV_i += P_bar_i^T dO_i | S_{i+1} | dK_i += dS_i^T Q_i | dQ_i = dS_i K | dP_{i+1}
 // Barrier phases run on per-CTA counters, so items follow one another without
 // re-initialisation: `g` counts query-tile steps, `n_done` counts items.
-template <int D>
+// E: the element format (ElemBF16 or ElemF16) of Q, K, V, dO, dK, dV and of
+// the P_bar and dS operands.
+template <int D, typename E = ElemBF16>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -352,9 +356,9 @@ __global__ void __launch_bounds__(512, 1)
     } else if (warp == 13) {
       // ---------------------------------------------------------- MMA issuer
       if (lane == 0) {
-        constexpr uint32_t kIdS = make_idesc_bf16(128, 128, 0, 0);   // K Q^T, V dO^T: K-major operands
-        constexpr uint32_t kIdAcc = make_idesc_bf16(128, D, 0, 1);   // TMEM A x MN-major B (dV, dK)
-        constexpr uint32_t kIdDQ = make_idesc_bf16(128, D, 1, 1);    // dS (MN-major) x K (MN-major)
+        constexpr uint32_t kIdS = make_idesc(128, 128, 0, 0, E::kMmaFmt);   // K Q^T, V dO^T: K-major operands
+        constexpr uint32_t kIdAcc = make_idesc(128, D, 0, 1, E::kMmaFmt);   // TMEM A x MN-major B (dV, dK)
+        constexpr uint32_t kIdDQ = make_idesc(128, D, 1, 1, E::kMmaFmt);    // dS (MN-major) x K (MN-major)
         // Descriptors as 32-bit low halves with one shared high half (every
         // operand has a 1024-byte stride): this thread shares its issue slots
         // with the busiest warps of the CTA, so each MMA costs it only an add.
@@ -505,7 +509,7 @@ __global__ void __launch_bounds__(512, 1)
                                        __uint_as_float(r[i >> 4][(2 * i + 1) & 31])),
                                c2, h ? f2_pack(nl.z, nl.w) : f2_pack(nl.x, nl.y)),
                         x0, x1);
-              pk[i] = pack_bf16(ex2(x0), ex2(x1));
+              pk[i] = E::pack(ex2(x0), ex2(x1));
             }
           }
           // masked keys (past N) and, on the diagonal tile, queries before the
@@ -553,13 +557,13 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int i = 2 * j + h;
-              const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[i]));
+              const float2 pp = E::unpack(pk[i]);
               const uint64_t dq2 = h ? f2_pack(d4.z, d4.w) : f2_pack(d4.x, d4.y);
               const uint64_t dp2 = f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
                                            __uint_as_float(r[i >> 4][(2 * i + 1) & 31]));
               float y0, y1;
               f2_unpack(f2_mul(f2_fma(dq2, f2_pack(-1.f, -1.f), dp2), f2_pack(pp.x, pp.y)), y0, y1);
-              dsw[i] = pack_bf16(y0, y1);
+              dsw[i] = E::pack(y0, y1);
             }
           }
         }
@@ -651,14 +655,15 @@ __global__ void __launch_bounds__(512, 1)
           tmem_ld_wait(r);
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            ov[c * 16 + i] = pack_bf16(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
+            ov[c * 16 + i] = E::pack(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
         }
         if (which == 1) {
           tc_fence_before();
           mbar_arrive(dkv_free);                     // the next item may overwrite dK, dV
         }
         if (key < p.N) {
-          uint4* dst = reinterpret_cast<uint4*>((which ? p.dk : p.dv) + (size_t(w.bh) * p.N + key) * D);
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<typename E::T*>(which ? p.dk : p.dv) +
+                                                (size_t(w.bh) * p.N + key) * D);
 #pragma unroll
           for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
         }

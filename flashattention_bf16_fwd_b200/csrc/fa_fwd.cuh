@@ -31,7 +31,7 @@
 namespace fa {
 
 struct FwdParams {
-  __nv_bfloat16* o;     // [BH, N, D]
+  void* o;              // [BH, N, D] of the element type
   float* lse;           // [BH, N]
   int32_t* ties;        // [BH, N] or nullptr
   int* dev_error;       // library error flag
@@ -91,9 +91,11 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
   return it;
 }
 
+// E: the element format (ElemBF16 or ElemF16) of Q, K, V, O and of P_bar.
 // kVariants: compiled with the code of fix_mode 4 (self-normalised) and 5
-// (near ties); the other instantiation, used for fix_mode 0-3, leaves it out.
-template <int D, bool kVariants>
+// (near ties, bf16 only); the other instantiation, used for fix_mode 0-3,
+// leaves it out.
+template <int D, bool kVariants, typename E = ElemBF16>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -197,8 +199,8 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == 9) {
       // ---------------------------------------------------------- MMA issuer
       if (lane == 0) {
-        constexpr uint32_t kIdS = make_idesc_bf16(128, 128, 0, 0);   // Q K^T: both K-major
-        constexpr uint32_t kIdPV = make_idesc_bf16(128, D, 0, 1);    // P_bar V: V is MN-major
+        constexpr uint32_t kIdS = make_idesc(128, 128, 0, 0, E::kMmaFmt);   // Q K^T: both K-major
+        constexpr uint32_t kIdPV = make_idesc(128, D, 0, 1, E::kMmaFmt);    // P_bar V: V is MN-major
         // Descriptors are built once; each MMA only advances the start address.
         const uint64_t dq0 = make_sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
         const uint64_t dk0 = make_sdesc_sw128(smem_u32(smem + L::kKVOff), 16, 1024);
@@ -395,7 +397,7 @@ __global__ void __launch_bounds__(384, 1)
         if (kVariants && p.near) {
           int cn = 0;
 #pragma unroll
-          for (int i = 0; i < 128; ++i) cn += (s[i] >= 0.998046875f) ? 1 : 0;
+          for (int i = 0; i < 128; ++i) cn += (s[i] >= 0.998046875f) ? 1 : 0;   // bf16: 1 - 2^-9
           cn_new = (m == m_new ? cnt_near : 0) + cn;
         }
         const int det = (kVariants && p.near) ? cn_new : c_new;
@@ -442,11 +444,13 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]);
+          for (int i = 0; i < 16; ++i) pk[i] = E::pack(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]);
           if (kVariants && p.self_norm) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              rs_bar += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
+            for (int i = 0; i < 16; ++i) {
+              const float2 pp = E::unpack(pk[i]);
+              rs_bar += pp.x + pp.y;
+            }
           }
           tmem_st16(t_p + c * 16, pk);
         }
@@ -492,13 +496,13 @@ __global__ void __launch_bounds__(384, 1)
         const float inv_l = 1.f / ((kVariants && p.self_norm) ? l_bar : l);
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          ow[c * 16 + i] = pack_bf16(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+          ow[c * 16 + i] = E::pack(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
       }
       // O_t is in registers: the next item's first P_bar V may overwrite it
       tc_fence_before();
       mbar_arrive(&o_free[t]);
       if (row < p.N) {
-        uint4* dst = reinterpret_cast<uint4*>(p.o + (size_t(w.bh) * p.N + row) * D);
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<typename E::T*>(p.o) + (size_t(w.bh) * p.N + row) * D);
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(ow[4 * i], ow[4 * i + 1], ow[4 * i + 2], ow[4 * i + 3]);
         p.lse[size_t(w.bh) * p.N + row] = (ms + (raised ? p.delta_log2 : 0.f) + lg2(l)) * kLn2;

@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace fa {
@@ -219,6 +220,12 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, int a_mn_ma
          (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
+// The same for an element format: 1 = bf16, 0 = f16 (A and B always share it).
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N, int a_mn_major, int b_mn_major, uint32_t fmt) {
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) |
+         (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (the layout a TMA box with
 // CU_TENSOR_MAP_SWIZZLE_128B and a 128-byte inner extent writes).
 //   bits 0-13 start >> 4, 16-29 leading byte offset >> 4, 32-45 stride byte
@@ -399,6 +406,13 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   return d;
 }
 
+// Two floats -> one 32-bit word of fp16 (round to nearest even), lo in bits 0-15.
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // Two floats -> one 32-bit word of bf16 (round to nearest even), lo in bits 0-15.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
@@ -436,5 +450,25 @@ __device__ __forceinline__ void regs_set() {
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+
+// The 16-bit element formats of the kernels: storage type, tcgen05 operand
+// format, and the conversions between a packed pair and two floats.
+struct ElemBF16 {
+  using T = __nv_bfloat16;
+  static constexpr uint32_t kMmaFmt = 1;
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi) { return pack_bf16(lo, hi); }
+  static __device__ __forceinline__ float2 unpack(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  }
+};
+
+struct ElemF16 {
+  using T = __half;
+  static constexpr uint32_t kMmaFmt = 0;
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi) { return pack_f16(lo, hi); }
+  static __device__ __forceinline__ float2 unpack(uint32_t w) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&w));
+  }
+};
 
 }  // namespace fa

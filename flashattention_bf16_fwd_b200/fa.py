@@ -13,7 +13,8 @@ import os
 import torch
 
 __all__ = [
-    "FAError", "LIB_PATH", "lib", "fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_bwd", "fa_bwd_gqa", "fa_bwd_workspace_size",
+    "FAError", "LIB_PATH", "lib", "fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_fwd_f16", "fa_bwd", "fa_bwd_gqa",
+    "fa_bwd_f16", "fa_bwd_workspace_size",
     "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc", "fa_watchdog_selftest",
     "fa_status_string", "fa_check_device_error", "EXPORTED", "attention_fwd", "attention_bwd",
 ]
@@ -21,7 +22,8 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
 
 FA_OK = 0
-EXPORTED = ("fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_bwd_gqa", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
+EXPORTED = ("fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_f16", "fa_bwd_f16", "fa_bwd_workspace_size",
+            "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
             "fa_bwd_finish", "fa_bwd_noalloc", "fa_watchdog_selftest", "fa_status_string",
             "fa_check_device_error")
 
@@ -43,6 +45,10 @@ def _load() -> ctypes.CDLL:
     so.fa_fwd.restype = i
     so.fa_fwd_ties.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     so.fa_fwd_ties.restype = i
+    so.fa_fwd_f16.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    so.fa_fwd_f16.restype = i
+    so.fa_bwd_f16.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, vp]
+    so.fa_bwd_f16.restype = i
     so.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
     so.fa_fwd_gqa.restype = i
     so.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, f, vp]
@@ -109,6 +115,19 @@ def fa_fwd_ties(q, k, v, o, lse, ties, causal: bool, scale: float, fix_mode: int
     B, H, N, d = _shape(q)
     return lib.fa_fwd_ties(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(ties), B, H, N, d, int(causal),
                            float(scale), int(fix_mode), _stream(stream))
+
+
+def fa_fwd_f16(q, k, v, o, lse, causal: bool, scale: float, fix_mode: int, stream=None) -> int:
+    B, H, N, d = _shape(q)
+    return lib.fa_fwd_f16(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, int(causal), float(scale),
+                          int(fix_mode), _stream(stream))
+
+
+def fa_bwd_f16(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool, scale: float, stream=None) -> int:
+    B, H, N, d = _shape(q)
+    return lib.fa_bwd_f16(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                          _ptr(workspace), _nbytes(workspace), B, H, N, d, int(causal), float(scale),
+                          _stream(stream))
 
 
 def fa_fwd_gqa(q, k, v, o, lse, causal: bool, scale: float, fix_mode: int, stream=None) -> int:

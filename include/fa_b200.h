@@ -113,6 +113,22 @@ FA_API int fa_fwd_ties(const void* q, const void* k, const void* v, void* o, flo
                 float scale, int fix_mode, void* stream);
 
 /*
+ * FP16 variant: Q, K, V, O, dO, dQ, dK, dV are fp16 [B,H,N,d] instead of bf16
+ * (the pages treat FP16 and BF16 together as the low-precision formats of the
+ * instability).  P_bar is rounded to fp16; the fix (fix_mode 1) maps repeated
+ * maxima to 1 - 2^-11, the largest fp16 value below 1.  fix_mode must be 0 or
+ * 1 (FA_ERR_FIXMODE otherwise).  Arguments, layouts and the workspace are as
+ * in fa_fwd / fa_bwd.
+ */
+FA_API int fa_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse,
+                      int B, int H, int N, int d, int causal, float scale, int fix_mode,
+                      void* stream);
+FA_API int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o,
+                      const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                      void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                      int causal, float scale, void* stream);
+
+/*
  * Grouped-query attention (GQA; MQA when Hkv == 1), the head layout of the
  * larger Llama 2 models the chibakuma.com page names: H query heads share Hkv
  * key/value heads, query head h reading key/value head h / (H / Hkv).

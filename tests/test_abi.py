@@ -31,7 +31,7 @@ def declared_symbols():
 
 
 def test_header_declares_the_boundary():
-    assert declared_symbols() == sorted(["fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_bwd_gqa",
+    assert declared_symbols() == sorted(["fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_f16", "fa_bwd_f16",
                                          "fa_bwd_workspace_size", "fa_bwd",
                                          "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish",
                                          "fa_bwd_noalloc", "fa_watchdog_selftest", "fa_status_string",
@@ -109,6 +109,16 @@ def test_bwd_argument_errors(fa):
 
 
 FA_ERR_SCRATCH_LIMIT = -11
+
+
+def test_f16_argument_errors(fa):
+    # the fp16 path carries fix_mode 0 and 1 only
+    assert fa.lib.fa_fwd_f16(A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 2, None) == FA_ERR_FIXMODE
+    assert fa.lib.fa_fwd_f16(A, A, A, A, None, 1, 1, 128, 64, 1, 0.125, 1, None) == FA_ERR_NULL
+    assert fa.lib.fa_fwd_f16(A, A, A, A, A, 1, 1, 128, 96, 1, 0.125, 1, None) == FA_ERR_HEADDIM
+    ws = fa.fa_bwd_workspace_size(1, 1, 128, 64)
+    assert fa.lib.fa_bwd_f16(A, A, A, A, A, A, MIS, A, A, A, ws, 1, 1, 128, 64, 1, 0.125, None) == FA_ERR_ALIGN
+    assert fa.lib.fa_bwd_f16(A, A, A, A, A, A, A, A, A, A, ws - 1, 1, 1, 128, 64, 1, 0.125, None) == FA_ERR_WORKSPACE
 
 
 def test_gqa_argument_errors(fa):
