@@ -379,9 +379,12 @@ def measured_traffic(kernel, w):
         rec = json.load(f).get(kernel)
     if not rec:
         return None
+    # the hash covers the sources the kernel is compiled from (all of csrc/
+    # when the record names none)
     src = os.path.join(ROOT, "flashattention_bf16_fwd_b200", "csrc")
+    files = rec.get("sources") or sorted(os.listdir(src))
     h = hashlib.sha256()
-    for fn in sorted(os.listdir(src)):
+    for fn in files:
         with open(os.path.join(src, fn), "rb") as f:
             h.update(f.read())
     if rec.get("csrc_sha256") != h.hexdigest():
