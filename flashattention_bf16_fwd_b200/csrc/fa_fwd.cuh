@@ -371,39 +371,26 @@ __global__ void __launch_bounds__(384, 1)
         const float ms_new = (m_new == kNegInf) ? 0.f : m_new * sl2;
 
         // A row whose running maximum is already repeated and does not move in
-        // this tile keeps the raised shift whatever the tile holds: its P takes
-        // the factor 2^-delta in the loop below (times 1 on every other row),
-        // and only rows that become repeated in this tile need the rare path.
+        // this tile keeps the raised shift whatever the tile holds, so its P
+        // is computed with the raised shift directly (the exponent minus delta:
+        // any maximum in this tile rounds to 1 - 2^-8 in bf16 all the same).
+        // Only rows that become repeated in this tile need the rare path.
         const bool raise_early = p.fix && m == m_new && ((kVariants && p.near) ? cnt_near : cnt) >= 2;
-        // P = 2^(S*scale_log2 - ms_new); the row sum and the count of entries
+        const float msh = raise_early ? ms_new + p.delta_log2 : ms_new;
+        // P = 2^(S*scale_log2 - shift); the row sum and the count of entries
         // equal to the tile max ride along as independent packed adds
         uint64_t sum2[4] = {0, 0, 0, 0};
         uint64_t eq2[2] = {0, 0};
-        if (__any_sync(0xffffffffu, raise_early)) {
-          const uint64_t f2_early = raise_early ? f2_pack(kFixFactor, kFixFactor) : f2_pack(1.f, 1.f);
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const float x0 = fmaf(s[2 * i], sl2, -ms_new);
-            const float x1 = fmaf(s[2 * i + 1], sl2, -ms_new);
-            const float e0 = (s[2 * i] == mt) ? 1.f : 0.f;
-            const float e1 = (s[2 * i + 1] == mt) ? 1.f : 0.f;
-            eq2[i & 1] = f2_add(eq2[i & 1], f2_pack(e0, e1));
-            const uint64_t p2 = f2_mul(f2_pack(ex2(x0), ex2(x1)), f2_early);
-            f2_unpack(p2, s[2 * i], s[2 * i + 1]);
-            sum2[i & 3] = f2_add(sum2[i & 3], p2);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const float x0 = fmaf(s[2 * i], sl2, -ms_new);
-            const float x1 = fmaf(s[2 * i + 1], sl2, -ms_new);
-            const float e0 = (s[2 * i] == mt) ? 1.f : 0.f;
-            const float e1 = (s[2 * i + 1] == mt) ? 1.f : 0.f;
-            eq2[i & 1] = f2_add(eq2[i & 1], f2_pack(e0, e1));
-            s[2 * i] = ex2(x0);
-            s[2 * i + 1] = ex2(x1);
-            sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(s[2 * i], s[2 * i + 1]));
-          }
+        for (int i = 0; i < 64; ++i) {
+          const float x0 = fmaf(s[2 * i], sl2, -msh);
+          const float x1 = fmaf(s[2 * i + 1], sl2, -msh);
+          const float e0 = (s[2 * i] == mt) ? 1.f : 0.f;
+          const float e1 = (s[2 * i + 1] == mt) ? 1.f : 0.f;
+          eq2[i & 1] = f2_add(eq2[i & 1], f2_pack(e0, e1));
+          s[2 * i] = ex2(x0);
+          s[2 * i + 1] = ex2(x1);
+          sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(s[2 * i], s[2 * i + 1]));
         }
         float ea, eb;
         f2_unpack(f2_add(eq2[0], eq2[1]), ea, eb);
