@@ -77,6 +77,11 @@ def test_fwd_argument_errors(fa):
     assert fwd(fa, N=0) == FA_ERR_SHAPE
     assert fwd(fa, B=0) == FA_ERR_SHAPE
     assert fwd(fa, B=1 << 14, H=1 << 10, N=1 << 10, d=64) == FA_ERR_SHAPE
+    # the bound is B*H*N*d < 2^31: 32768 heads of 1024 x 64 is exactly 2^31
+    assert fwd(fa, H=32768, N=1024, d=64) == FA_ERR_SHAPE
+    assert fwd(fa, H=32767, N=1024, d=64) == FA_ERR_DEVICE     # passes the checks; no GPU here
+    assert fa.fa_bwd_workspace_size(1, 32768, 1024, 64) == 0
+    assert fa.fa_bwd_workspace_size(1, 32767, 1024, 64) == 32767 * 1024 * (64 + 1) * 4
     assert fwd(fa, causal=2) == FA_ERR_ARG
     assert fwd(fa, scale=0.0) == FA_ERR_ARG
     assert fwd(fa, scale=float("nan")) == FA_ERR_ARG

@@ -207,6 +207,45 @@ def test_full_size_sampled_heads(fa, name):
         assert torch.isfinite(t).all()
 
 
+def test_largest_allowed_size(fa):
+    """The ABI's size bound: B*H*N*d one head short of 2^31 elements.
+
+    32767 heads of N=1024, d=64 (2^31 - 65536 elements, 4.3 GB per bf16
+    tensor).  The first head and the last, whose elements lie just below the
+    2^31-element offset, carry seeded oracle inputs and must match the oracle;
+    every other head holds seeded N(0, 1) values and every output must be
+    finite.  Catches any 32-bit element or byte offset in the kernels, the
+    tensor maps and the workspace split."""
+    N, d = 1024, 64
+    BH = 2 ** 31 // (N * d) - 1
+    assert BH * N * d < 2 ** 31 <= (BH + 1) * N * d
+    free, _ = torch.cuda.mem_get_info()
+    if free < 64 * 2 ** 30:
+        pytest.skip(f"needs 64 GiB of free device memory, {free / 2 ** 30:.0f} GiB free")
+    dev = torch.device("cuda")
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(31)
+    shape = (1, BH, N, d)
+    t = {n: torch.randn(shape, generator=gen, device=dev, dtype=torch.bfloat16) for n in ("q", "k", "v", "do")}
+    one = Workload("edge", 1, 1, N, d)
+    ends = {0: make_inputs(one, seed=41), BH - 1: make_inputs(one, seed=42)}
+    for h, x in ends.items():
+        for n in t:
+            t[n][:, h:h + 1] = x[n].to(dev)
+    o, lse = fa.attention_fwd(t["q"], t["k"], t["v"], causal=True, scale=one.scale, fix_mode=1)
+    dq, dk, dv = fa.attention_bwd(t["q"], t["k"], t["v"], o, lse, t["do"], causal=True, scale=one.scale)
+    torch.cuda.synchronize()
+    assert fa.fa_check_device_error() == 0
+    for h, x in ends.items():
+        g = {n: r[:, h:h + 1].float().cpu().numpy() for n, r in dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv).items()}
+        check_fwd(g, x)
+        check_bwd(g, x)
+    for r in (o, lse, dq, dk, dv):
+        assert torch.isfinite(r).all()
+    del t, o, lse, dq, dk, dv
+    torch.cuda.empty_cache()
+
+
 def test_no_sign_coherent_bias_with_fix(fa):
     """Repeated-max rows: the fix leaves no sign-coherent error in O.
 
