@@ -88,12 +88,20 @@ def barrier(world):
 
 
 def all_max(x: float, world: int) -> float:
+    """The largest of the ranks' values (every rank gets it): the slowest rank's time."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_tflops(world: int, steps: int, flops_per_step: float, t_max_ms: float) -> float:
+    """Whole-job throughput of `world` replicas that each ran `steps` steps: the
+    work of all ranks divided by the slowest rank's time."""
+    return world * steps * flops_per_step / (t_max_ms * 1e-3) / 1e12
 
 
 class ClockSampler:
@@ -309,7 +317,7 @@ def run_ours(args, rank, world, local):
     t_max = all_max(t_rank, world)
     outer_ms = all_max(outer[0].elapsed_time(outer[1]), world)
     flops = workload_flops(w.B, w.H, w.N, w.d, w.causal)
-    value = world * args.steps * flops["total"] / (t_max * 1e-3) / 1e12
+    value = replica_tflops(world, args.steps, flops["total"], t_max)
 
     peaks, peak_kind = load_peaks()
     kern_names = ["fa_fwd_kernel", "fa_bwd_pre_kernel", "fa_bwd_kernel", "fa_bwd_dq_kernel"]
@@ -430,7 +438,7 @@ def run_e2e(fa, x, w, args, dev, stream, flops_total, world):
     t = all_max(ev[0].elapsed_time(ev[1]), world)
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    return {"value": world * steps * flops_total / (t * 1e-3) / 1e12, "unit": "TFLOP/s",
+    return {"value": replica_tflops(world, steps, flops_total, t), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": t / steps}
 
