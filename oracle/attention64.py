@@ -38,7 +38,9 @@ What it computes, and where each step is stated:
 * The same in FP16 (the pages treat FP16 and BF16 together as the
   low-precision formats of the instability: yicaiai article, abstract):
   P_bar rounded to fp16, and the fix maps the maxima to 1 - 2^-11, the
-  largest fp16 value below 1.
+  largest fp16 value below 1.  The variants carry over: fix_mode 2, 3 and 4
+  as above, fix_mode 5 with the near-tie test made in fp16 (P rounds to 1 in
+  fp16 when P >= 1 - 2^-12).
 * Grouped-query attention (GQA/MQA head layouts, the Llama 2 family the
   chibakuma.com page names): H_q query heads share H_kv key/value heads,
   query head h reading key/value head h // (H_q / H_kv).  The forward is the
@@ -57,7 +59,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "DELTA_LOG2", "DELTA_NAT", "DELTA16_NAT", "fp16_round", "FIX_SHIFT_NAT", "SELF_NORMALISED_MODES", "NEAR_TIE_MODES", "bf16_round", "scores", "attention_fwd",
+    "DELTA_LOG2", "DELTA_NAT", "DELTA16_NAT", "fp16_round", "FIX_SHIFT_NAT", "FIX_SHIFT_NAT_FP16", "SELF_NORMALISED_MODES", "NEAR_TIE_MODES", "bf16_round", "scores", "attention_fwd",
     "attention_bwd", "attention_fwd_bf16p", "tie_counts", "near_tie_counts", "gqa_expand", "gqa_reduce",
 ]
 
@@ -76,6 +78,10 @@ _FP16_MAX = (2.0 - 2.0 ** -10) * 2.0 ** 15
 
 # The fix's shift for fp16 P_bar (natural-log units): maxima -> 1 - 2^-11.
 DELTA16_NAT = -np.log(1.0 - 2.0 ** -11)
+
+# FIX_SHIFT_NAT for fp16 P_bar: modes 1 and 5 land the maxima on 1 - 2^-11,
+# the largest fp16 value below 1; modes 2, 3 and 4 do not depend on the format.
+FIX_SHIFT_NAT_FP16 = {0: 0.0, 1: DELTA16_NAT, 2: float(np.log(2.0)), 3: 1.0 / 16.0, 4: 0.0, 5: DELTA16_NAT}
 
 
 def bf16_round(x) -> np.ndarray:
@@ -212,8 +218,10 @@ def gqa_reduce(x, group: int) -> np.ndarray:
     return x.reshape(B, H // group, group, N, d).sum(axis=2)
 
 
-def near_tie_counts(q, k, causal: bool, scale: float) -> np.ndarray:
-    """#{j visible : bf16(exp(scale * (S_ij - max_j S_ij))) == 1} per row."""
+def near_tie_counts(q, k, causal: bool, scale: float, fmt: str = "bf16") -> np.ndarray:
+    """#{j visible : round(exp(scale * (S_ij - max_j S_ij))) == 1} per row, the
+    rounding being to bf16 (default) or to fp16 (fmt = "fp16")."""
+    round_fn = {"bf16": bf16_round, "fp16": fp16_round}[fmt]
     q, k = _f64(q), _f64(k)
     B, H, N, _ = q.shape
     out = np.zeros((B, H, N), dtype=np.int64)
@@ -221,7 +229,7 @@ def near_tie_counts(q, k, causal: bool, scale: float) -> np.ndarray:
     for b, h in _heads(q):
         s = np.where(vis, scale * (q[b, h] @ k[b, h].T), -np.inf)
         p = np.exp(s - s.max(axis=1, keepdims=True))
-        out[b, h] = np.sum(bf16_round(p) == 1.0, axis=1)
+        out[b, h] = np.sum(round_fn(p) == 1.0, axis=1)
     return out
 
 
@@ -242,15 +250,16 @@ def attention_fwd_bf16p(q, k, v, causal: bool, scale: float, fix_mode: int,
     P_bar == 1 exactly; fix_mode 1 maps them to 1 - 2^-8, fix_mode 2 to 0.5,
     fix_mode 3 to exp(-1/16); fix_mode 4 keeps them at 1 and self-normalises;
     fix_mode 5 is fix_mode 1 triggered by near ties.
-    fmt = "fp16" rounds P_bar to fp16 instead (fix_mode 0 or 1 only; the fix
-    then maps the maxima to 1 - 2^-11).
+    fmt = "fp16" rounds P_bar to fp16 instead; fix_mode 1 and 5 then map the
+    maxima to 1 - 2^-11 (FIX_SHIFT_NAT_FP16), and fix_mode 5 counts the
+    entries whose P rounds to 1 in fp16.
     """
     if fix_mode not in FIX_SHIFT_NAT:
         raise ValueError("fix_mode must be 0, 1, 2, 3, 4 or 5")
-    if fmt not in ("bf16", "fp16") or (fmt == "fp16" and fix_mode not in (0, 1)):
-        raise ValueError("fmt must be bf16, or fp16 with fix_mode 0 or 1")
+    if fmt not in ("bf16", "fp16"):
+        raise ValueError("fmt must be bf16 or fp16")
     round_fn = bf16_round if fmt == "bf16" else fp16_round
-    shifts = FIX_SHIFT_NAT if fmt == "bf16" else {0: 0.0, 1: DELTA16_NAT}
+    shifts = FIX_SHIFT_NAT if fmt == "bf16" else FIX_SHIFT_NAT_FP16
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, N, d = q.shape
     o = np.empty((B, H, N, v.shape[-1]))

@@ -233,6 +233,71 @@ def fp16_pins(M):
             ok &= np.array_equal(torch.from_numpy(r1).to(torch.float16).double().numpy(), r1)
     if not ok:
         failed.append("fp16_fix_property")
+    # the variants with fp16 P_bar: where the maxima of a repeated-max row land,
+    # unrounded and after the fp16 rounding.  exp(-1/16) = 0.9394130..., and
+    # 2^11 times that is 1923.918..., so fp16 rounds it to 1924 / 2048.
+    for fix, top, top16 in ((2, 0.5, 0.5), (3, float(np.exp(-1.0 / 16.0)), 1924.0 / 2048.0)):
+        _, _, pu = M.attention_fwd_bf16p(q, k, v, True, 0.5, fix, round_p=False, return_pbar=True, fmt="fp16")
+        _, _, pr = M.attention_fwd_bf16p(q, k, v, True, 0.5, fix, return_pbar=True, fmt="fp16")
+        ok = True
+        for h in range(2):
+            for i in range(q.shape[2]):
+                ru, rr = pu[0, h, i, : i + 1], pr[0, h, i, : i + 1]
+                if ties[h, i] >= 2:
+                    ok &= abs(ru.max() - top) <= 1e-15 and np.sum(np.abs(ru - top) <= 1e-15) == ties[h, i]
+                    ok &= rr.max() == top16
+                else:
+                    ok &= ru.max() == 1.0 and rr.max() == 1.0
+        if not ok:
+            failed.append(f"fp16_variant_maxima_fix{fix}")
+    # self-normalised with fp16 P_bar: V = 1 gives O = 1 exactly
+    o4, _ = M.attention_fwd_bf16p(q, k, np.ones_like(v), True, 0.5, 4, fmt="fp16")
+    if not np.allclose(o4, 1.0, atol=1e-14, rtol=0):
+        failed.append("fp16_self_normalised_ones")
+    # near ties in fp16: every query is (2, 0), key 2 is key 0 moved by a gap
+    # g in its first coordinate, so from row 2 on the maximum is key 2 and key
+    # 0 trails it by g in S.  Head 0: g = 1e-4, P = exp(-g) rounds to 1 in fp16
+    # and in bf16.  Head 1: g = 1e-3, P rounds to 1 in bf16 (>= 1 - 2^-9) but
+    # not in fp16 (< 1 - 2^-12).  Counts by brute force (math.exp, torch's
+    # casts), then fix_mode 5's property with fp16 P_bar.
+    n = 7
+    qn = np.zeros((1, 2, n, 2))
+    qn[..., 0] = 2.0
+    kn = np.zeros((1, 2, n, 2))
+    kn[0, :, 0] = (1.0, 0.0)
+    kn[0, :, 1] = (0.0, 1.0)
+    kn[0, :, 3:] = (0.5, 0.0)
+    kn[0, 0, 2] = (1.0 + 1e-4, 0.0)
+    kn[0, 1, 2] = (1.0 + 1e-3, 0.0)
+    vn = rng.standard_normal((1, 2, n, 3))
+    sc = 0.5
+    brute16 = np.zeros((1, 2, n), dtype=np.int64)
+    brute_bf = np.zeros((1, 2, n), dtype=np.int64)
+    exact = np.zeros((1, 2, n), dtype=np.int64)
+    for h in range(2):
+        for i in range(n):
+            row = [sc * sum(qn[0, h, i, c] * kn[0, h, j, c] for c in range(qn.shape[3])) for j in range(i + 1)]
+            mx = max(row)
+            pr = torch.tensor([math.exp(r - mx) for r in row], dtype=torch.float64).float()
+            brute16[0, h, i] = int((pr.to(torch.float16).float() == 1.0).sum())
+            brute_bf[0, h, i] = int((pr.to(torch.bfloat16).float() == 1.0).sum())
+            exact[0, h, i] = sum(r == mx for r in row)
+    if not np.array_equal(M.near_tie_counts(qn, kn, True, sc, fmt="fp16"), brute16):
+        failed.append("fp16_near_tie_counts")
+    if not (np.any((brute16 >= 2) & (exact < 2)) and np.any(brute16 != brute_bf)):
+        failed.append("fp16_near_tie_fixture")
+    _, _, p5 = M.attention_fwd_bf16p(qn, kn, vn, True, sc, 5, return_pbar=True, fmt="fp16")
+    _, _, p0 = M.attention_fwd_bf16p(qn, kn, vn, True, sc, 0, return_pbar=True, fmt="fp16")
+    ok = True
+    for h in range(2):
+        for i in range(n):
+            r5, r0 = p5[0, h, i, : i + 1], p0[0, h, i, : i + 1]
+            if brute16[0, h, i] >= 2:
+                ok &= bool(np.all(r5 < 1.0)) and np.sum(r0 == 1.0) == brute16[0, h, i]
+            else:
+                ok &= np.array_equal(r5, r0)
+    if not ok:
+        failed.append("fp16_near_tie_fix_property")
     return failed
 
 
@@ -491,20 +556,25 @@ MUTATIONS = [
     ("fix_wrong_delta", "DELTA_NAT = -np.log(1.0 - 2.0 ** -8)", "DELTA_NAT = -np.log(1.0 - 2.0 ** -6)"),
     ("emulation_skips_rounding", "pbar = round_fn(p) if round_p else p", "pbar = p"),
     ("ties_ignore_mask", "s = np.where(vis, q[b, h] @ k[b, h].T, -np.inf)\n        out[b, h]", "s = q[b, h] @ k[b, h].T\n        out[b, h]"),
-    ("variant_shift_in_log2", "2: float(np.log(2.0))", "2: 1.0"),
-    ("variant_off_grid_value", "3: 1.0 / 16.0", "3: 1.0 / 8.0"),
+    ("variant_shift_in_log2", "1: DELTA_NAT, 2: float(np.log(2.0))", "1: DELTA_NAT, 2: 1.0"),
+    ("variant_off_grid_value", "3: 1.0 / 16.0, 4: 0.0, 5: DELTA_NAT}", "3: 1.0 / 8.0, 4: 0.0, 5: DELTA_NAT}"),
     ("self_normalised_unrounded_den", "den = pbar.sum(axis=1, keepdims=True) if", "den = l if"),
     ("near_ties_count_exact_ties", "ties = np.sum(round_fn(np.exp(s - m)) == 1.0, axis=1, keepdims=True)",
      "ties = np.sum(raw == raw.max(axis=1, keepdims=True), axis=1, keepdims=True)"),
     ("near_tie_no_shift", "4: 0.0, 5: DELTA_NAT}", "4: 0.0, 5: 0.0}"),
-    ("near_tie_threshold_off", "out[b, h] = np.sum(bf16_round(p) == 1.0, axis=1)", "out[b, h] = np.sum(p == 1.0, axis=1)"),
+    ("near_tie_threshold_off", "out[b, h] = np.sum(round_fn(p) == 1.0, axis=1)", "out[b, h] = np.sum(p == 1.0, axis=1)"),
     ("gqa_expand_wrong_axis", "return np.repeat(_f64(x), group, axis=1)", "return np.tile(_f64(x), (1, group, 1, 1))"),
     ("gqa_reduce_mean", "return x.reshape(B, H // group, group, N, d).sum(axis=2)",
      "return x.reshape(B, H // group, group, N, d).mean(axis=2)"),
     ("fp16_one_bit_short", "q_exp = np.maximum(e, -13) - 11", "q_exp = np.maximum(e, -13) - 10"),
     ("fp16_no_subnormals", "q_exp = np.maximum(e, -13) - 11", "q_exp = e - 11"),
-    ("fp16_fix_bf16_delta", "shifts = FIX_SHIFT_NAT if fmt == \"bf16\" else {0: 0.0, 1: DELTA16_NAT}",
+    ("fp16_fix_bf16_delta", "shifts = FIX_SHIFT_NAT if fmt == \"bf16\" else FIX_SHIFT_NAT_FP16",
      "shifts = FIX_SHIFT_NAT"),
+    ("fp16_variant_shift_in_log2", "1: DELTA16_NAT, 2: float(np.log(2.0))", "1: DELTA16_NAT, 2: 1.0"),
+    ("fp16_variant_off_grid_value", "3: 1.0 / 16.0, 4: 0.0, 5: DELTA16_NAT}", "3: 1.0 / 8.0, 4: 0.0, 5: DELTA16_NAT}"),
+    ("fp16_near_tie_no_shift", "4: 0.0, 5: DELTA16_NAT}", "4: 0.0, 5: 0.0}"),
+    ("fp16_near_tie_rounds_in_bf16", "round_fn = {\"bf16\": bf16_round, \"fp16\": fp16_round}[fmt]",
+     "round_fn = bf16_round"),
     ("self_normalised_lse_from_pbar", "lse[b, h] = shift[:, 0] + np.log(l[:, 0])",
      "lse[b, h] = shift[:, 0] + np.log(den[:, 0])"),
 ]
