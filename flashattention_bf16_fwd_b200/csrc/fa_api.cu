@@ -75,6 +75,8 @@ DeviceState* device_state() {
     setup(fa_fwd_kernel<128, true, ElemBF16>, FwdLayout<128>::kAlloc, FwdLayout<128>::kLaunchRegs);
     setup(fa_fwd_kernel<64, false, ElemF16>, FwdLayout<64>::kAlloc, FwdLayout<64>::kLaunchRegs);
     setup(fa_fwd_kernel<128, false, ElemF16>, FwdLayout<128>::kAlloc, FwdLayout<128>::kLaunchRegs);
+    setup(fa_fwd_kernel<64, true, ElemF16>, FwdLayout<64>::kAlloc, FwdLayout<64>::kLaunchRegs);
+    setup(fa_fwd_kernel<128, true, ElemF16>, FwdLayout<128>::kAlloc, FwdLayout<128>::kLaunchRegs);
     setup(fa_bwd_kernel<64, ElemBF16>, BwdLayout<64>::kAlloc, BwdLayout<64>::kLaunchRegs);
     setup(fa_bwd_kernel<128, ElemBF16>, BwdLayout<128>::kAlloc, BwdLayout<128>::kLaunchRegs);
     setup(fa_bwd_kernel<64, ElemF16>, BwdLayout<64>::kAlloc, BwdLayout<64>::kLaunchRegs);
@@ -169,7 +171,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if (rc != FA_OK) return rc;
   if ((rc = check_heads(H, Hkv)) != FA_OK) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGN;
-  if (fix_mode < 0 || fix_mode > (kF16 ? 1 : 5)) return FA_ERR_FIXMODE;
+  if (fix_mode < 0 || fix_mode > 5) return FA_ERR_FIXMODE;
   DeviceState* st = device_state();
   if (!st) return FA_ERR_DEVICE;
   const int BH = B * H;
@@ -191,9 +193,9 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   prm.causal = causal;
   prm.scale_log2 = float(double(scale) * 1.4426950408889634);
   // shift on repeated-max rows per fix_mode, in base-2 units: 1 and 5 map the
-  // maxima to 1 - 2^-8, 2 to 0.5, 3 to exp(-1/16); 0 and 4 keep the plain shift
-  const double delta = (fix_mode == 1 && kF16)           ? kDeltaLog2F16
-                       : (fix_mode == 1 || fix_mode == 5) ? kDeltaLog2
+  // maxima to the largest value below 1 of the P_bar format (1 - 2^-8 in bf16,
+  // 1 - 2^-11 in fp16), 2 to 0.5, 3 to exp(-1/16); 0 and 4 keep the plain shift
+  const double delta = (fix_mode == 1 || fix_mode == 5) ? (kF16 ? kDeltaLog2F16 : kDeltaLog2)
                        : fix_mode == 2                  ? 1.0
                        : fix_mode == 3                  ? 1.4426950408889634 / 16.0
                                                         : 0.0;
@@ -205,8 +207,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   const int n_items = prm.n_pairs * BH;
   const dim3 grid(unsigned(n_items < st->num_sms ? n_items : st->num_sms));
   const bool variants = fix_mode >= 4;   // self-normalised or near-tie code
-  auto kern = (d == 64) ? (variants ? fa_fwd_kernel<64, !kF16, E> : fa_fwd_kernel<64, false, E>)
-                        : (variants ? fa_fwd_kernel<128, !kF16, E> : fa_fwd_kernel<128, false, E>);
+  auto kern = (d == 64) ? (variants ? fa_fwd_kernel<64, true, E> : fa_fwd_kernel<64, false, E>)
+                        : (variants ? fa_fwd_kernel<128, true, E> : fa_fwd_kernel<128, false, E>);
   const int smem = (d == 64) ? FwdLayout<64>::kAlloc : FwdLayout<128>::kAlloc;
   const cudaError_t e = launch(kern, grid, dim3(FwdLayout<64>::kThreads), smem, stream, mq, mk, mv, prm);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
@@ -413,6 +415,28 @@ int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o, const
                            scale, stream);
 }
 
+int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties, int B, int H,
+              int Hkv, int N, int d, int causal, float scale, int fix_mode, int elem, void* stream) {
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (elem == FA_ELEM_BF16)
+    return launch_fwd<ElemBF16>(q, k, v, o, lse, ties, B, H, Hkv, N, d, causal, scale, fix_mode, s);
+  if (elem == FA_ELEM_F16)
+    return launch_fwd<ElemF16>(q, k, v, o, lse, ties, B, H, Hkv, N, d, causal, scale, fix_mode, s);
+  return FA_ERR_ARG;
+}
+
+int fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+              void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N,
+              int d, int causal, float scale, int elem, void* stream) {
+  if (elem == FA_ELEM_BF16)
+    return bwd_impl<ElemBF16>(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, N, d,
+                              causal, scale, stream);
+  if (elem == FA_ELEM_F16)
+    return bwd_impl<ElemF16>(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, N, d,
+                             causal, scale, stream);
+  return FA_ERR_ARG;
+}
+
 const char* fa_status_string(int status) {
   switch (status) {
     case FA_OK: return "ok";
@@ -424,7 +448,9 @@ const char* fa_status_string(int status) {
     case FA_ERR_WORKSPACE: return "workspace is NULL, misaligned or smaller than fa_bwd_workspace_size()";
     case FA_ERR_LAUNCH: return "the CUDA runtime refused a kernel launch";
     case FA_ERR_TIMEOUT: return "a kernel gave up on a bounded wait (device error flag set)";
-    case FA_ERR_ARG: return "causal must be 0 or 1 and scale finite and > 0";
+    case FA_ERR_ARG:
+      return "an argument is out of range: causal not 0 or 1, scale not finite and > 0, elem not an fa_elem "
+             "value, or a watchdog timeout outside 1..1000000 us";
     case FA_ERR_DEVICE: return "no sm_100 device, or tensor-map encoding unavailable";
     case FA_ERR_SCRATCH_LIMIT:
       return "fa_bwd_noalloc: fa_bwd_workspace_size() exceeds FA_BWD_NOALLOC_SCRATCH_BYTES (32 MiB)";

@@ -22,7 +22,7 @@
 // gives back down to 88 and the two softmax warpgroups take 208 each:
 // 128 * (208 + 208 + 88) = 384 * 168.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 after.
-// P_bar (bf16, two per 32-bit column) overwrites the first 64 columns of S_t
+// P_bar (bf16 or fp16, two per 32-bit column) overwrites the first 64 columns of S_t
 // and is the A operand of O_t += P_bar V (V is the MN-major B operand).
 #pragma once
 
@@ -39,10 +39,10 @@ struct FwdParams {
   int H, group;         // query heads per batch entry; query heads per K/V head (1 = no sharing)
   float scale_log2;     // scale * log2(e): S -> base-2 exponent domain
   float delta_log2;     // shift added to m on repeated-max rows (0 = fix off)
-  float fix_factor;     // 2^-delta_log2: P at a repeated maximum (1 - 2^-8, 0.5 or exp(-1/16))
+  float fix_factor;     // 2^-delta_log2: P at a repeated maximum (1 - 2^-8 or, in fp16, 1 - 2^-11; 0.5; exp(-1/16))
   int fix;              // raise the shift on repeated-max rows
   int self_norm;        // divide O by the sum of the rounded P_bar instead of the unrounded P
-  int near;             // detect near ties (P rounds to bf16 1.0) instead of exact ties of S
+  int near;             // detect near ties (P rounds to 1.0 in the element format) instead of exact ties of S
 };
 
 template <int D>
@@ -93,8 +93,7 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
 
 // E: the element format (ElemBF16 or ElemF16) of Q, K, V, O and of P_bar.
 // kVariants: compiled with the code of fix_mode 4 (self-normalised) and 5
-// (near ties, bf16 only); the other instantiation, used for fix_mode 0-3,
-// leaves it out.
+// (near ties); the other instantiation, used for fix_mode 0-3, leaves it out.
 template <int D, bool kVariants, typename E = ElemBF16>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -316,7 +315,8 @@ __global__ void __launch_bounds__(384, 1)
     const float sl2 = p.scale_log2;
     // 2^-delta: on a repeated-max row P is computed with the plain shift and
     // then multiplied by this, which is the same as raising m by delta; each
-    // maximum lands on this value (1 - 2^-8 for fix_mode 1).
+    // maximum lands on this value (1 - 2^-8 for fix_mode 1 in bf16, 1 - 2^-11
+    // in fp16).
     const float kFixFactor = p.fix_factor;
     uint32_t it_cnt = 0;   // softmax iterations done by this warpgroup
     bool ok = true;
@@ -373,7 +373,8 @@ __global__ void __launch_bounds__(384, 1)
         // A row whose running maximum is already repeated and does not move in
         // this tile keeps the raised shift whatever the tile holds, so its P
         // is computed with the raised shift directly (the exponent minus delta:
-        // any maximum in this tile rounds to 1 - 2^-8 in bf16 all the same).
+        // any maximum in this tile rounds to 2^-delta on the P_bar grid all the
+        // same).
         // Only rows that become repeated in this tile need the rare path.
         const bool raise_early = p.fix && m == m_new && ((kVariants && p.near) ? cnt_near : cnt) >= 2;
         const float msh = raise_early ? ms_new + p.delta_log2 : ms_new;
@@ -398,13 +399,13 @@ __global__ void __launch_bounds__(384, 1)
         int c_new = (m == m_new ? cnt : 0) + (mt == m_new ? ct : 0);
         if (m_new == kNegInf) c_new = 0;
         // near-tie mode: entries of this tile whose P (plain shift) rounds to
-        // bf16 1.0, i.e. P >= 1 - 2^-9; earlier tiles' count stands while the
-        // shift has not moved
+        // 1.0 in the element format (P >= 1 - 2^-9 in bf16, 1 - 2^-12 in
+        // fp16); earlier tiles' count stands while the shift has not moved
         int cn_new = 0;
         if (kVariants && p.near) {
           int cn = 0;
 #pragma unroll
-          for (int i = 0; i < 128; ++i) cn += (s[i] >= 0.998046875f) ? 1 : 0;   // bf16: 1 - 2^-9
+          for (int i = 0; i < 128; ++i) cn += (s[i] >= E::kRoundsToOne) ? 1 : 0;
           cn_new = (m == m_new ? cnt_near : 0) + cn;
         }
         const int det = (kVariants && p.near) ? cn_new : c_new;

@@ -14,7 +14,7 @@ import torch
 
 __all__ = [
     "FAError", "LIB_PATH", "lib", "fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_fwd_f16", "fa_bwd", "fa_bwd_gqa",
-    "fa_bwd_f16", "fa_bwd_workspace_size",
+    "fa_bwd_f16", "fa_fwd_ex", "fa_bwd_ex", "FA_ELEM_BF16", "FA_ELEM_F16", "fa_bwd_workspace_size",
     "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc", "fa_watchdog_selftest",
     "fa_status_string", "fa_check_device_error", "EXPORTED", "attention_fwd", "attention_bwd",
 ]
@@ -22,7 +22,9 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
 
 FA_OK = 0
-EXPORTED = ("fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_f16", "fa_bwd_f16", "fa_bwd_workspace_size",
+FA_ELEM_BF16, FA_ELEM_F16 = 0, 1
+EXPORTED = ("fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_f16", "fa_bwd_f16", "fa_fwd_ex", "fa_bwd_ex",
+            "fa_bwd_workspace_size",
             "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
             "fa_bwd_finish", "fa_bwd_noalloc", "fa_watchdog_selftest", "fa_status_string",
             "fa_check_device_error")
@@ -53,6 +55,10 @@ def _load() -> ctypes.CDLL:
     so.fa_fwd_gqa.restype = i
     so.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, f, vp]
     so.fa_bwd_gqa.restype = i
+    so.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+    so.fa_fwd_ex.restype = i
+    so.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, f, i, vp]
+    so.fa_bwd_ex.restype = i
     so.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     so.fa_bwd_workspace_size.restype = sz
     so.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, vp]
@@ -145,6 +151,29 @@ def fa_bwd_gqa(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool, scale: 
                           _stream(stream))
 
 
+def _elem(t) -> int:
+    if t.dtype == torch.bfloat16:
+        return FA_ELEM_BF16
+    if t.dtype == torch.float16:
+        return FA_ELEM_F16
+    raise ValueError(f"tensors must be bfloat16 or float16, not {t.dtype}")
+
+
+def fa_fwd_ex(q, k, v, o, lse, ties, causal: bool, scale: float, fix_mode: int, stream=None) -> int:
+    """The general forward: element format from q's dtype, Hkv from k's head count, ties optional."""
+    B, H, N, d = _shape(q)
+    return lib.fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(ties), B, H, int(k.shape[1]), N, d,
+                         int(causal), float(scale), int(fix_mode), _elem(q), _stream(stream))
+
+
+def fa_bwd_ex(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool, scale: float, stream=None) -> int:
+    """The general backward: element format from q's dtype, Hkv from k's head count."""
+    B, H, N, d = _shape(q)
+    return lib.fa_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                         _ptr(workspace), _nbytes(workspace), B, H, int(k.shape[1]), N, d, int(causal),
+                         float(scale), _elem(q), _stream(stream))
+
+
 def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
     return int(lib.fa_bwd_workspace_size(B, H, N, d))
 
@@ -197,28 +226,49 @@ def _check(call: str, status: int):
         raise FAError(call, status)
 
 
+def _validate(q, k, v, like_q=()):
+    """Shapes, dtypes, devices and contiguity the C ABI assumes but cannot see:
+    q and like_q [B,H,N,d]; k, v [B,Hkv,N,d] with Hkv dividing H; one dtype."""
+    B, H, N, d = _shape(q)
+    if k.dim() != 4 or k.shape[0] != B or tuple(k.shape[2:]) != (N, d) or v.shape != k.shape:
+        raise ValueError(f"k and v must be [B, Hkv, N, d] = [{B}, Hkv, {N}, {d}], got {tuple(k.shape)}, "
+                         f"{tuple(v.shape)}")
+    if H % int(k.shape[1]) != 0:
+        raise ValueError(f"the {k.shape[1]} key/value heads must divide the {H} query heads")
+    for t in like_q:
+        if t.shape != q.shape:
+            raise ValueError(f"expected a {tuple(q.shape)} tensor, got {tuple(t.shape)}")
+    for t in (q, k, v) + tuple(like_q):
+        if t.dtype != q.dtype or t.device != q.device or not t.is_contiguous():
+            raise ValueError("q, k, v, o and do must share one dtype and device and be contiguous")
+
+
 def attention_fwd(q, k, v, causal: bool = True, scale: float | None = None, fix_mode: int = 1,
                   stream=None, ties: bool = False):
-    """Allocate O and LSE (and optionally the per-row tie counts) and run fa_fwd."""
+    """Allocate O and LSE (and optionally the per-row tie record) and run the
+    forward.  bf16 or fp16 tensors (from q's dtype); k and v may have fewer
+    heads than q (grouped-query attention)."""
+    _validate(q, k, v)
     B, H, N, d = _shape(q)
     scale = d ** -0.5 if scale is None else scale
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if ties:
-        t = torch.empty((B, H, N), dtype=torch.int32, device=q.device)
-        _check("fa_fwd_ties", fa_fwd_ties(q, k, v, o, lse, t, causal, scale, fix_mode, stream))
-        return o, lse, t
-    _check("fa_fwd", fa_fwd(q, k, v, o, lse, causal, scale, fix_mode, stream))
-    return o, lse
+    t = torch.empty((B, H, N), dtype=torch.int32, device=q.device) if ties else None
+    _check("fa_fwd_ex", fa_fwd_ex(q, k, v, o, lse, t, causal, scale, fix_mode, stream))
+    return (o, lse, t) if ties else (o, lse)
 
 
 def attention_bwd(q, k, v, o, lse, do, causal: bool = True, scale: float | None = None, stream=None,
                   workspace=None):
-    """Allocate dQ, dK, dV (and the workspace unless given) and run fa_bwd."""
+    """Allocate dQ, dK, dV (and the workspace unless given) and run the
+    backward.  Formats and head layout as in attention_fwd."""
+    _validate(q, k, v, (o, do))
     B, H, N, d = _shape(q)
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
     scale = d ** -0.5 if scale is None else scale
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if workspace is None:
         workspace = torch.empty(fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=q.device)
-    _check("fa_bwd", fa_bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal, scale, stream))
+    _check("fa_bwd_ex", fa_bwd_ex(q, k, v, o, lse, do, dq, dk, dv, workspace, causal, scale, stream))
     return dq, dk, dv

@@ -62,7 +62,8 @@ typedef enum {
   FA_ERR_WORKSPACE = -6, /* workspace NULL, misaligned or too small           */
   FA_ERR_LAUNCH = -7,    /* the CUDA runtime refused a launch                 */
   FA_ERR_TIMEOUT = -8,   /* a kernel's bounded wait expired (device flag)     */
-  FA_ERR_ARG = -9,       /* causal not in {0,1}, or scale not finite and > 0  */
+  FA_ERR_ARG = -9,       /* causal not in {0,1}, scale not finite and > 0, or
+                            elem not an fa_elem value                         */
   FA_ERR_DEVICE = -10,   /* no sm_100 device, or the driver entry point for
                             tensor maps is unavailable                        */
   FA_ERR_SCRATCH_LIMIT = -11 /* fa_bwd_noalloc: the problem needs more scratch
@@ -115,9 +116,10 @@ FA_API int fa_fwd_ties(const void* q, const void* k, const void* v, void* o, flo
 /*
  * FP16 variant: Q, K, V, O, dO, dQ, dK, dV are fp16 [B,H,N,d] instead of bf16
  * (the pages treat FP16 and BF16 together as the low-precision formats of the
- * instability).  P_bar is rounded to fp16; the fix (fix_mode 1) maps repeated
- * maxima to 1 - 2^-11, the largest fp16 value below 1.  fix_mode must be 0 or
- * 1 (FA_ERR_FIXMODE otherwise).  Arguments, layouts and the workspace are as
+ * instability).  P_bar is rounded to fp16.  The fix modes carry over with the
+ * fp16 grid: 1 and 5 map repeated maxima to 1 - 2^-11, the largest fp16 value
+ * below 1; 2, 3 and 4 are as in fa_fwd; 5 counts entries whose P rounds to
+ * fp16 1.0, i.e. P >= 1 - 2^-12.  Arguments, layouts and the workspace are as
  * in fa_fwd / fa_bwd.
  */
 FA_API int fa_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -146,6 +148,27 @@ FA_API int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o
                       const float* lse, const void* dout, void* dq, void* dk, void* dv,
                       void* workspace, size_t workspace_bytes, int B, int H, int Hkv,
                       int N, int d, int causal, float scale, void* stream);
+
+/* Element formats of fa_fwd_ex / fa_bwd_ex. */
+typedef enum { FA_ELEM_BF16 = 0, FA_ELEM_F16 = 1 } fa_elem;
+
+/*
+ * fa_fwd_ex / fa_bwd_ex - one call for every combination of the above: the
+ * element format `elem` (FA_ELEM_BF16 or FA_ELEM_F16) of every [.,.,N,d]
+ * tensor and of P_bar, H query heads over Hkv key/value heads (Hkv == H:
+ * ordinary attention), any fix_mode 0-5, and the optional `ties` record of
+ * fa_fwd_ties (NULL to skip it).  fa_fwd, fa_fwd_ties, fa_fwd_f16, fa_fwd_gqa
+ * and the matching backward calls are this call with their fixed arguments.
+ * Layouts, ownership, the workspace and the error codes are theirs;
+ * FA_ERR_ARG also reports an unknown elem.
+ */
+FA_API int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int32_t* ties, int B, int H, int Hkv, int N, int d, int causal,
+                     float scale, int fix_mode, int elem, void* stream);
+FA_API int fa_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                     void* workspace, size_t workspace_bytes, int B, int H, int Hkv,
+                     int N, int d, int causal, float scale, int elem, void* stream);
 
 /*
  * fa_bwd_workspace_size - bytes of device scratch fa_bwd needs:

@@ -32,7 +32,7 @@ def declared_symbols():
 
 def test_header_declares_the_boundary():
     assert declared_symbols() == sorted(["fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_f16", "fa_bwd_f16",
-                                         "fa_bwd_workspace_size", "fa_bwd",
+                                         "fa_fwd_ex", "fa_bwd_ex", "fa_bwd_workspace_size", "fa_bwd",
                                          "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish",
                                          "fa_bwd_noalloc", "fa_watchdog_selftest", "fa_status_string",
                                          "fa_check_device_error"])
@@ -116,9 +116,46 @@ def test_bwd_argument_errors(fa):
 FA_ERR_SCRATCH_LIMIT = -11
 
 
+def test_general_entry_point_argument_errors(fa):
+    fx = lambda **kw: fa.lib.fa_fwd_ex(*[kw.get(n, dflt) for n, dflt in (
+        ("q", A), ("k", A), ("v", A), ("o", A), ("lse", A), ("ties", None), ("B", 1), ("H", 4), ("Hkv", 2),
+        ("N", 128), ("d", 64), ("causal", 1), ("scale", 0.125), ("fix", 1), ("elem", 0), ("stream", None))])
+    assert fx() == FA_ERR_DEVICE                      # valid arguments, no GPU here
+    assert fx(elem=1, fix=5) == FA_ERR_DEVICE
+    assert fx(elem=2) == FA_ERR_ARG
+    assert fx(elem=-1) == FA_ERR_ARG
+    assert fx(fix=6) == FA_ERR_FIXMODE
+    assert fx(Hkv=3) == FA_ERR_SHAPE
+    assert fx(v=None) == FA_ERR_NULL
+    assert fx(o=MIS, elem=1) == FA_ERR_ALIGN
+    ws = fa.fa_bwd_workspace_size(1, 4, 128, 64)
+    bx = lambda **kw: fa.lib.fa_bwd_ex(*[kw.get(n, dflt) for n, dflt in (
+        ("q", A), ("k", A), ("v", A), ("o", A), ("lse", A), ("do", A), ("dq", A), ("dk", A), ("dv", A),
+        ("ws", A), ("wsz", ws), ("B", 1), ("H", 4), ("Hkv", 2), ("N", 128), ("d", 64), ("causal", 1),
+        ("scale", 0.125), ("elem", 1), ("stream", None))])
+    assert bx() == FA_ERR_DEVICE
+    assert bx(elem=3) == FA_ERR_ARG
+    assert bx(wsz=ws - 1) == FA_ERR_WORKSPACE
+    assert bx(Hkv=8) == FA_ERR_SHAPE
+    assert bx(d=96) == FA_ERR_HEADDIM
+
+
+def test_binding_checks_shapes_and_dtypes(fa):
+    q = torch.zeros(1, 4, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):                   # k with a head count that does not divide H
+        fa.attention_fwd(q, torch.zeros(1, 3, 128, 64, dtype=torch.bfloat16), torch.zeros(1, 3, 128, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):                   # mixed element formats
+        fa.attention_fwd(q, q.half(), q)
+    with pytest.raises(ValueError):                   # not contiguous
+        fa.attention_fwd(q.transpose(2, 3).contiguous().transpose(2, 3), q, q)
+    with pytest.raises(ValueError):                   # float32 is not a supported format
+        fa.attention_fwd(q.float(), q.float(), q.float())
+
+
 def test_f16_argument_errors(fa):
-    # the fp16 path carries fix_mode 0 and 1 only
-    assert fa.lib.fa_fwd_f16(A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 2, None) == FA_ERR_FIXMODE
+    # the fp16 path carries every fix_mode, 0-5
+    assert fa.lib.fa_fwd_f16(A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 6, None) == FA_ERR_FIXMODE
+    assert fa.lib.fa_fwd_f16(A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 5, None) == FA_ERR_DEVICE   # no GPU here
     assert fa.lib.fa_fwd_f16(A, A, A, A, None, 1, 1, 128, 64, 1, 0.125, 1, None) == FA_ERR_NULL
     assert fa.lib.fa_fwd_f16(A, A, A, A, A, 1, 1, 128, 96, 1, 0.125, 1, None) == FA_ERR_HEADDIM
     ws = fa.fa_bwd_workspace_size(1, 1, 128, 64)
