@@ -12,9 +12,10 @@ import numpy as np
 import pytest
 import torch
 
-from flashattention_bf16_fwd_b200.stats import lse_rel_err, normwise_rel_err
+from flashattention_bf16_fwd_b200.stats import bias_stats, lse_rel_err, normwise_rel_err
 from flashattention_bf16_fwd_b200.workloads import WORKLOADS, make_inputs
-from oracle import attention_bwd, attention_fwd, attention_fwd_bf16p, gqa_expand, gqa_reduce, near_tie_counts
+from oracle import (attention_bwd, attention_fwd, attention_fwd_bf16p, gqa_expand, gqa_reduce, near_tie_counts,
+                    tie_counts)
 
 pytestmark = pytest.mark.gpu
 
@@ -103,6 +104,25 @@ def test_f16_self_normalised_output_of_ones(fa):
     assert np.abs(o4 - 1.0).max() <= 2.0 ** -11          # one fp16 step below 1 at most
     assert np.mean(o4 == 1.0) > 0.99
 
+
+
+def test_f16_bias_sweep_over_fix_modes(fa):
+    """The bias statistics of every mode with fp16 P_bar on the repeated-max
+    rows of the long-structured input (printed).  As in bf16, fix_mode 1 must
+    show no sign-coherent error (|z| < 3 for both statistics)."""
+    w = WORKLOADS["long"].with_shape(B=2, H=8, N=2048)
+    x = make_inputs(w, seed=1, with_grad=False)
+    q, k, v = (x[n].half() for n in ("q", "k", "v"))
+    o_ref, _ = attention_fwd(q, k, v, True, w.scale)
+    rep = tie_counts(q, k, True) >= 2
+    assert rep.sum() > 1000
+    rows = {}
+    for mode in range(6):
+        o, _, _ = fwd(fa, q, k, v, True, w.scale, mode)
+        rows[mode] = s = bias_stats(o, o_ref, rep)
+        print(f"fp16 fix_mode {mode}: z_mean {s['z_mean']:+.2f}  z_aligned {s['z_aligned']:+.2f}  "
+              f"aligned_mean/mean|O| {s['aligned_mean'] / s['mean_abs_ref']:+.3e}")
+    assert abs(rows[1]["z_mean"]) < 3 and abs(rows[1]["z_aligned"]) < 3
 
 GQA_CASES = [(1, 4, 2, 300, 64, True, 1), (2, 8, 1, 256, 128, True, 5), (1, 6, 3, 384, 64, False, 3)]
 
