@@ -91,6 +91,13 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
   return it;
 }
 
+// The smallest value below 1 that rounds to 1.0 in E's format (ties to even):
+// 1 - 2^-9 in bf16, 1 - 2^-12 in fp16.  P at or above it gives P_bar == 1.
+template <typename E>
+__device__ __forceinline__ constexpr float rounds_to_one() {
+  return E::kMmaFmt == 1 ? 0.998046875f : 0.999755859375f;
+}
+
 // E: the element format (ElemBF16 or ElemF16) of Q, K, V, O and of P_bar.
 // kVariants: compiled with the code of fix_mode 4 (self-normalised) and 5
 // (near ties); the other instantiation, used for fix_mode 0-3, leaves it out.
@@ -405,7 +412,7 @@ __global__ void __launch_bounds__(384, 1)
         if (kVariants && p.near) {
           int cn = 0;
 #pragma unroll
-          for (int i = 0; i < 128; ++i) cn += (s[i] >= E::kRoundsToOne) ? 1 : 0;
+          for (int i = 0; i < 128; ++i) cn += (s[i] >= rounds_to_one<E>()) ? 1 : 0;
           cn_new = (m == m_new ? cnt_near : 0) + cn;
         }
         const int det = (kVariants && p.near) ? cn_new : c_new;
