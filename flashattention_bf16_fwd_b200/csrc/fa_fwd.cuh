@@ -320,10 +320,11 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t t_p = tmem + lane_base + L::tm_p(t);
     const uint32_t t_o = tmem + lane_base + L::tm_o(t);
     const float sl2 = p.scale_log2;
-    // 2^-delta: on a repeated-max row P is computed with the plain shift and
-    // then multiplied by this, which is the same as raising m by delta; each
-    // maximum lands on this value (1 - 2^-8 for fix_mode 1 in bf16, 1 - 2^-11
-    // in fp16).
+    // 2^-delta: on a row whose maximum becomes repeated in the current tile,
+    // P is computed with the plain shift and then multiplied by this, which is
+    // the same as raising m by delta (rows repeated before the tile take the
+    // raised shift in the exponent instead); each maximum lands on this value
+    // (1 - 2^-8 for fix_mode 1 in bf16, 1 - 2^-11 in fp16).
     const float kFixFactor = p.fix_factor;
     uint32_t it_cnt = 0;   // softmax iterations done by this warpgroup
     bool ok = true;
