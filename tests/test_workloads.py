@@ -3,7 +3,7 @@ import numpy as np
 import torch
 
 from flashattention_bf16_fwd_b200.workloads import WORKLOADS, make_inputs, workload_flops
-from oracle import tie_counts
+from oracle import near_tie_counts, tie_counts
 
 
 def test_deterministic_by_seed():
@@ -33,6 +33,21 @@ def test_sink_and_key_dup_structures_tie():
     x = make_inputs(lg, seed=0, with_grad=False)
     assert np.mean(tie_counts(x["q"], x["k"], True) >= 2) > 0.01
 
+
+
+def test_argmax_near_has_near_ties_and_no_exact_ties():
+    """The near-tie structure: every constructed copy scores one bf16 step of
+    one key element below the maximum, so no row ties exactly, and a large
+    share of rows has two or more P that round to 1 (bf16).  Rounding to 1 in
+    fp16 (P >= 1 - 2^-12) implies it in bf16 (P >= 1 - 2^-9), so the fp16
+    near-tie rows are a subset of the bf16 ones."""
+    for seed in (0, 3):
+        x = make_inputs(WORKLOADS["tiny"].with_shape(structure="argmax_near"), seed=seed, with_grad=False)
+        assert not np.any(tie_counts(x["q"], x["k"], True) >= 2)
+        near = near_tie_counts(x["q"], x["k"], True, x["scale"]) >= 2
+        near16 = near_tie_counts(x["q"].half(), x["k"].half(), True, x["scale"], fmt="fp16") >= 2
+        assert near.mean() > 0.25 and near16.mean() > 0.15, (near.mean(), near16.mean())
+        assert not np.any(near16 & ~near)
 
 def test_flop_convention():
     f = workload_flops(8, 12, 1024, 64, True)
