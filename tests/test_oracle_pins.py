@@ -254,6 +254,12 @@ def fp16_pins(M):
     o4, _ = M.attention_fwd_bf16p(q, k, np.ones_like(v), True, 0.5, 4, fmt="fp16")
     if not np.allclose(o4, 1.0, atol=1e-14, rtol=0):
         failed.append("fp16_self_normalised_ones")
+    # LSE stays the unrounded log-sum-exp of the definition in every mode
+    _, lse_exact = M.attention_fwd(q, k, v, True, 0.5)
+    for fix in range(6):
+        _, le = M.attention_fwd_bf16p(q, k, v, True, 0.5, fix, fmt="fp16")
+        if not np.allclose(le, lse_exact, atol=1e-13, rtol=0):
+            failed.append(f"fp16_lse_unrounded_fix{fix}")
     # near ties in fp16: every query is (2, 0), key 2 is key 0 moved by a gap
     # g in its first coordinate, so from row 2 on the maximum is key 2 and key
     # 0 trails it by g in S.  Head 0: g = 1e-4, P = exp(-g) rounds to 1 in fp16
