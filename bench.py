@@ -14,7 +14,17 @@ with programmatic dependent launch); the L2 is flushed (a 512 MiB write)
 before each step, outside the events.  A second pass of the same number of
 steps calls the backward's three launches one by one with events between all
 four kernels: it gives the per-kernel times and the roofline of the dominant
-kernel.  Multi-GPU runs are independent replicas (attention over (B, H) has no
+kernel.  A third pass repeats the first without the flush (L2-warm).
+
+The line's headline is the chosen workload.  Its ``per_config`` block repeats
+the same three passes for each workload of ``--configs`` (default: GPT-2
+small, GPT-2 medium, the long-context shape and the Llama-2-7B shape), each
+over a step count sized to about a second: median step time flushed and
+warm, TFLOP/s, percent of peak, per-kernel times and the dominant kernel's
+roofline fraction, and at d = 64 the bound the MUFU exponentials put on the
+throughput.
+
+Multi-GPU runs are independent replicas (attention over (B, H) has no
 exchange step): each rank runs the full workload on its own GPU, and the
 slowest rank's time is used.
 """
@@ -46,7 +56,7 @@ L2_FLUSH_BYTES = 512 << 20
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt2s")
@@ -55,6 +65,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", default="gpt2s,gpt2m,long,llama7b",
+                    help="workloads measured into the line's per_config block (comma list, or none)")
     return ap.parse_args()
 
 
@@ -240,88 +252,99 @@ def workload_config(w, args):
             "parallelism": "replicas", "l2": "flushed before every step (512 MiB write, outside the events)"}
 
 
-def run_ours(args, rank, world, local):
-    from flashattention_bf16_fwd_b200 import fa
+KERNELS = ["fa_fwd_kernel", "fa_bwd_pre_kernel", "fa_bwd_kernel", "fa_bwd_dq_kernel"]
+# nominal MUFU ex2 throughput of one SM (results per clock), for the bound the
+# exponentials put on the d = 64 configurations
+MUFU_EX2_PER_CLK_PER_SM = 16
 
-    w = WORKLOADS[args.workload]
-    dev = torch.device("cuda", local if world > 1 else 0)
-    x = make_inputs(w, seed=args.seed + rank)
-    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
-    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
-    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
-    ws = torch.empty(fa.fa_bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    causal, scale, fix = w.causal, w.scale, args.fix_mode
 
-    def check(rc, what):
-        if rc != 0:
-            raise RuntimeError(f"{what}: {fa.fa_status_string(rc)}")
+def computed_tiles(N: int, causal: bool) -> int:
+    """128 x 128 score tiles a head computes (causal: the key tiles up to the
+    diagonal of each query tile, the diagonal's masked half included)."""
+    n = (N + 127) // 128
+    return n * (n + 1) // 2 if causal else n * n
 
-    def step_api():
-        check(fa.fa_fwd(q, k, v, o, lse, causal, scale, fix, stream), "fa_fwd")
-        check(fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal, scale, stream), "fa_bwd")
 
-    def step(ev):
-        ev[0].record(stream)
-        check(fa.fa_fwd(q, k, v, o, lse, causal, scale, fix, stream), "fa_fwd")
-        ev[1].record(stream)
-        check(fa.fa_bwd_preprocess(o, do, ws, stream), "fa_bwd_preprocess")
-        ev[2].record(stream)
-        check(fa.fa_bwd_main(q, k, v, lse, do, dk, dv, ws, causal, scale, stream), "fa_bwd_main")
-        ev[3].record(stream)
-        check(fa.fa_bwd_finish(dq, ws, scale, stream), "fa_bwd_finish")
-        ev[4].record(stream)
+def mufu_bound(w, sm_mhz: float, n_sms: int) -> dict:
+    """TFLOP/s the exponentials allow if MUFU ex2 were the only limit: one
+    exponential per computed score in the forward, one in the backward."""
+    exps = computed_tiles(w.N, w.causal) * 128 * 128 * w.B * w.H
+    rate = MUFU_EX2_PER_CLK_PER_SM * n_sms * sm_mhz * 1e6
+    fl = workload_flops(w.B, w.H, w.N, w.d, w.causal)
+    return {"fwd_tflops": fl["fwd"] / (exps / rate) / 1e12, "fwd_bwd_tflops": fl["total"] / (2 * exps / rate) / 1e12,
+            "ex2_per_clk_per_sm": MUFU_EX2_PER_CLK_PER_SM, "sm_mhz": sm_mhz, "exps_per_pass": exps,
+            "basis": "nominal MUFU rate x the SM clock sampled during the run"}
 
-    launches_per_step = 4
-    warm = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
-    for _ in range(max(args.warmup, 0)):
-        flush.zero_()
-        step_api()
-        flush.zero_()
-        step(warm)
+
+class Problem:
+    """One workload's inputs and outputs resident on the device."""
+
+    def __init__(self, fa, w, seed, dev, stream):
+        self.fa, self.w, self.stream = fa, w, stream
+        self.x = make_inputs(w, seed=seed)
+        self.q, self.k, self.v, self.do = (self.x[n].to(dev) for n in ("q", "k", "v", "do"))
+        self.o, self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(4))
+        self.lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(fa.fa_bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+
+    def step_api(self, fix):
+        fa, w = self.fa, self.w
+        check(fa.fa_fwd(self.q, self.k, self.v, self.o, self.lse, w.causal, w.scale, fix, self.stream), "fa_fwd")
+        check(fa.fa_bwd(self.q, self.k, self.v, self.o, self.lse, self.do, self.dq, self.dk, self.dv, self.ws,
+                        w.causal, w.scale, self.stream), "fa_bwd")
+
+    def step_split(self, fix, ev):
+        fa, w, s = self.fa, self.w, self.stream
+        ev[0].record(s)
+        check(fa.fa_fwd(self.q, self.k, self.v, self.o, self.lse, w.causal, w.scale, fix, s), "fa_fwd")
+        ev[1].record(s)
+        check(fa.fa_bwd_preprocess(self.o, self.do, self.ws, s), "fa_bwd_preprocess")
+        ev[2].record(s)
+        check(fa.fa_bwd_main(self.q, self.k, self.v, self.lse, self.do, self.dk, self.dv, self.ws, w.causal,
+                             w.scale, s), "fa_bwd_main")
+        ev[3].record(s)
+        check(fa.fa_bwd_finish(self.dq, self.ws, w.scale, s), "fa_bwd_finish")
+        ev[4].record(s)
+
+    def free(self):
+        for n in ("q", "k", "v", "do", "o", "dq", "dk", "dv", "lse", "ws"):
+            setattr(self, n, None)
+
+
+def check(rc, what):
+    if rc != 0:
+        from flashattention_bf16_fwd_b200 import fa
+        raise RuntimeError(f"{what}: {fa.fa_status_string(rc)}")
+
+
+def time_steps(pb, fix, steps, flush, stream):
+    """Per-step times (ms): one event pair around fa_fwd + fa_bwd on the
+    launching stream; with `flush`, a write larger than the L2 before each
+    step, outside the events."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    for i in range(steps):
+        if flush is not None:
+            flush.zero_()
+        ev[i][0].record(stream)
+        pb.step_api(fix)
+        ev[i][1].record(stream)
     torch.cuda.synchronize()
-    check(fa.fa_check_device_error(), "warm-up")
+    return np.array([a.elapsed_time(b) for a, b in ev])
 
-    # timed pass: one event pair per step, the kernels of a step back to back
-    bounds = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    sampler = ClockSampler(local if world > 1 else 0)
-    sampler.start()
-    time.sleep(0.2)
-    barrier(world)
-    torch.cuda.synchronize()
-    sampler.mark(True)
-    outer[0].record(stream)
-    for i in range(args.steps):
-        flush.zero_()
-        bounds[i][0].record(stream)
-        step_api()
-        bounds[i][1].record(stream)
-    outer[1].record(stream)
-    torch.cuda.synchronize()
-    # per-kernel pass: events between the four kernels of every step
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.zero_()
-        step(events[i])
-    torch.cuda.synchronize()
-    sampler.mark(False)
-    barrier(world)
-    clocks = sampler.stop()
-    check(fa.fa_check_device_error(), "timed steps")
 
-    step_ms = np.array([b[0].elapsed_time(b[1]) for b in bounds])
-    per = np.array([[events[i][j].elapsed_time(events[i][j + 1]) for j in range(4)] for i in range(args.steps)])
-    t_rank = float(step_ms.sum())
-    t_max = all_max(t_rank, world)
-    outer_ms = all_max(outer[0].elapsed_time(outer[1]), world)
+def time_kernels(pb, fix, steps, flush, stream):
+    """Per-kernel times (ms, [steps, 4]): events between the four launches."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        pb.step_split(fix, ev[i])
+    torch.cuda.synchronize()
+    return np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(4)] for i in range(steps)])
+
+
+def kernel_table(w, kern_ms, peaks, peak_kind):
+    """Per-kernel times, rates and the roofline of the dominant kernel."""
     flops = workload_flops(w.B, w.H, w.N, w.d, w.causal)
-    value = replica_tflops(world, args.steps, flops["total"], t_max)
-
-    peaks, peak_kind = load_peaks()
-    kern_names = ["fa_fwd_kernel", "fa_bwd_pre_kernel", "fa_bwd_kernel", "fa_bwd_dq_kernel"]
-    kern_ms = per.mean(axis=0)
     rows = w.B * w.H * w.N
     elem = rows * w.d
     work = {
@@ -331,26 +354,104 @@ def run_ours(args, rank, world, local):
         "fa_bwd_dq_kernel": ("hbm", elem * 4 + elem * 2),
     }
     kernels = {}
-    for name, ms in zip(kern_names, kern_ms):
+    for name, ms in zip(KERNELS, kern_ms):
         bound, amount = work[name]
         rate = amount / (ms * 1e-3)
         kernels[name] = {"ms": float(ms), "share": float(ms / kern_ms.sum()),
                          ("TFLOP/s" if bound == "tensor" else "GB/s"): rate / (1e12 if bound == "tensor" else 1e9)}
-    dom = kern_names[int(np.argmax(kern_ms))]
+    dom = KERNELS[int(np.argmax(kern_ms))]
     bound, amount = work[dom]
+    ms = kern_ms[KERNELS.index(dom)]
     if bound == "tensor":
-        achieved, peak, unit = amount / (kern_ms[kern_names.index(dom)] * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        achieved, peak, unit = amount / (ms * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
     else:
-        achieved, peak, unit = amount / (kern_ms[kern_names.index(dom)] * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
-    traffic = measured_traffic(dom, w)
+        achieved, peak, unit = amount / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
     roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_kind} burst",
+                "frac": achieved / peak, "traffic": measured_traffic(dom, w), "peak_source": f"{peak_kind} burst",
                 "algorithmic": amount,
                 "timing": "mean of the kernel's event-bracketed launches in the per-kernel pass"}
+    return kernels, roofline
+
+
+def run_ours(args, rank, world, local):
+    from flashattention_bf16_fwd_b200 import fa
+
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local if world > 1 else 0)
+    stream = torch.cuda.current_stream(dev)
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    fix = args.fix_mode
+    pb = Problem(fa, w, args.seed + rank, dev, stream)
+
+    warm = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        pb.step_api(fix)
+        flush.zero_()
+        pb.step_split(fix, warm)
+    torch.cuda.synchronize()
+    check(fa.fa_check_device_error(), "warm-up")
+
+    sampler = ClockSampler(local if world > 1 else 0)
+    sampler.start()
+    time.sleep(0.2)
+    # timed pass: one event pair per step, the kernels of a step back to back
+    outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.mark(True)
+    outer[0].record(stream)
+    step_ms = time_steps(pb, fix, args.steps, flush, stream)
+    outer[1].record(stream)
+    torch.cuda.synchronize()
+    per = time_kernels(pb, fix, args.steps, flush, stream)
+    warm_ms = time_steps(pb, fix, args.steps, None, stream)
+    barrier(world)
+    check(fa.fa_check_device_error(), "timed steps")
+
+    t_rank = float(step_ms.sum())
+    t_max = all_max(t_rank, world)
+    outer_ms = all_max(outer[0].elapsed_time(outer[1]), world)
+    flops = workload_flops(w.B, w.H, w.N, w.d, w.causal)
+    value = replica_tflops(world, args.steps, flops["total"], t_max)
+    peaks, peak_kind = load_peaks()
+    kernels, roofline = kernel_table(w, per.mean(axis=0), peaks, peak_kind)
+
+    # every other workload of the configuration list, same procedure
+    per_config = {}
+    names = [] if args.configs == "none" else [c for c in args.configs.split(",") if c]
+    for name in names:
+        if name == w.name:
+            res = {"step_ms_flushed": float(np.median(step_ms)), "step_ms_warm": float(np.median(warm_ms)),
+                   "steps": args.steps, "kern_ms": per.mean(axis=0), "workload": w}
+        else:
+            res = measure_config(fa, WORKLOADS[name], args, rank, dev, stream, flush)
+        per_config[name] = res
+    sampler.mark(False)
+    clocks = sampler.stop()
+    check(fa.fa_check_device_error(), "configurations")
+    sm_mhz = clocks.get("sm_mhz") or 1965.0
+    for name, res in per_config.items():
+        cw = res.pop("workload")
+        kern_ms = res.pop("kern_ms")
+        fl = workload_flops(cw.B, cw.H, cw.N, cw.d, cw.causal)["total"]
+        ktab, kroof = kernel_table(cw, kern_ms, peaks, peak_kind)
+        res.update({
+            "shape": f"B={cw.B} H={cw.H} N={cw.N} d={cw.d} {'causal' if cw.causal else 'full'}, {cw.structure}",
+            "tflops_flushed": fl / (res["step_ms_flushed"] * 1e-3) / 1e12,
+            "tflops_warm": fl / (res["step_ms_warm"] * 1e-3) / 1e12,
+        })
+        res["pct_of_measured_peak_flushed"] = res["tflops_flushed"] / peaks["bf16_tflops"] * 100.0
+        res["pct_of_datasheet_peak_flushed"] = res["tflops_flushed"] / DATASHEET_BF16_TFLOPS * 100.0
+        res["kernels"] = ktab
+        res["roofline"] = kroof
+        if cw.d == 64:
+            res["mufu_bound"] = mufu_bound(cw, sm_mhz, n_sms)
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(fa, x, w, args, dev, stream, flops["total"], world)
+        e2e = run_e2e(fa, pb.x, w, args, dev, stream, flops["total"], world)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -359,15 +460,20 @@ def run_ours(args, rank, world, local):
         "pct_of_peak": {"measured_burst": value / world / peaks["bf16_tflops"] * 100.0,
                         "datasheet": value / world / DATASHEET_BF16_TFLOPS * 100.0, "peak_source": peak_kind},
         "ms_per_step_bracket": outer_ms / args.steps,
+        "ms_per_step_warm_l2": float(np.median(warm_ms)),
         "ms_per_step_kernel_sum": float(per.sum(axis=1).mean()),
-        "roofline": roofline, "kernels": kernels, "gpu_launches": launches_per_step * args.steps,
+        "roofline": roofline, "kernels": kernels, "gpu_launches": len(KERNELS) * args.steps,
         "clocks": clocks,
     }
+    if w.d == 64:
+        line["mufu_bound"] = mufu_bound(w, sm_mhz, n_sms)
+    if per_config:
+        line["per_config"] = per_config
     if e2e is not None:
         line["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gout = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
-        fl, secs, heads, errs = oracle_sample(x, w, args.cpu_seconds, seed=args.seed, gpu_out=gout)
+        gout = {"o": pb.o, "lse": pb.lse, "dq": pb.dq, "dk": pb.dk, "dv": pb.dv}
+        fl, secs, heads, errs = oracle_sample(pb.x, w, args.cpu_seconds, seed=args.seed, gpu_out=gout)
         line["cpu_baseline"] = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
                                 "kind": "oracle",
                                 "sample": f"{len(heads)} of {w.B * w.H} (batch, head) pairs, FP64 NumPy "
@@ -375,6 +481,28 @@ def run_ours(args, rank, world, local):
         line["max_err"] = errs
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def measure_config(fa, w, args, rank, dev, stream, flush):
+    """Median step time of workload w with the L2 flushed and warm, and its
+    per-kernel times, each over a step count sized to about a second."""
+    pb = Problem(fa, w, args.seed + rank, dev, stream)
+    warm = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        pb.step_api(args.fix_mode)
+        flush.zero_()
+        pb.step_split(args.fix_mode, warm)
+    torch.cuda.synchronize()
+    est = max(warm[0].elapsed_time(warm[4]), 1e-3)
+    steps = int(min(args.steps, max(10, 1000.0 / est)))
+    flushed = time_steps(pb, args.fix_mode, steps, flush, stream)
+    per = time_kernels(pb, args.fix_mode, steps, flush, stream)
+    warm_ms = time_steps(pb, args.fix_mode, steps, None, stream)
+    pb.free()
+    torch.cuda.empty_cache()
+    return {"step_ms_flushed": float(np.median(flushed)), "step_ms_warm": float(np.median(warm_ms)),
+            "steps": steps, "kern_ms": per.mean(axis=0), "workload": w}
 
 
 def measured_traffic(kernel, w):

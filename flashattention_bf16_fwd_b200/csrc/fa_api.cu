@@ -26,7 +26,7 @@ constexpr int kMaxDevices = 64;
 
 struct DeviceState {
   std::once_flag once;
-  int ok = 0;            // 1 when the device is sm_100 and the flag address is known
+  int status = FA_ERR_DEVICE;   // FA_OK once the device passed every check below
   int num_sms = 0;
   int* dev_error = nullptr;
 };
@@ -48,8 +48,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 
 // Per-device set-up, done once with that device current: check the
 // architecture, opt the kernels into large shared memory, and resolve the
-// device address of the error flag.
-DeviceState* device_state() {
+// device address of the error flag.  Returns nullptr on failure; `why` (if
+// given) receives FA_ERR_DEVICE or FA_ERR_BUILD.
+DeviceState* device_state(int* why = nullptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   DeviceState* st = &g_devices[dev];
@@ -61,13 +62,15 @@ DeviceState* device_state() {
     if (cudaGetSymbolAddress(&addr, g_dev_error) != cudaSuccess) return;
     st->dev_error = static_cast<int*>(addr);
     bool ok = true;
+    bool regs_ok = true;
     // Every kernel instantiation: large shared memory, and the register count
     // at launch that its setmaxnreg split assumes (a miscounted pool would stall
-    // setmaxnreg.inc).
+    // setmaxnreg.inc, so a build whose count differs is refused as FA_ERR_BUILD).
     auto setup = [&](auto kernel, int smem, int regs) {
       cudaFuncAttributes fattr{};
       ok &= cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-      ok &= cudaFuncGetAttributes(&fattr, kernel) == cudaSuccess && fattr.numRegs == regs;
+      ok &= cudaFuncGetAttributes(&fattr, kernel) == cudaSuccess;
+      regs_ok &= fattr.numRegs == regs;
     };
     setup(fa_fwd_kernel<64, false, ElemBF16>, FwdLayout<64>::kAlloc, FwdLayout<64>::kLaunchRegs);
     setup(fa_fwd_kernel<128, false, ElemBF16>, FwdLayout<128>::kAlloc, FwdLayout<128>::kLaunchRegs);
@@ -81,10 +84,20 @@ DeviceState* device_state() {
     setup(fa_bwd_kernel<128, ElemBF16>, BwdLayout<128>::kAlloc, BwdLayout<128>::kLaunchRegs);
     setup(fa_bwd_kernel<64, ElemF16>, BwdLayout<64>::kAlloc, BwdLayout<64>::kLaunchRegs);
     setup(fa_bwd_kernel<128, ElemF16>, BwdLayout<128>::kAlloc, BwdLayout<128>::kLaunchRegs);
-    st->ok = ok ? 1 : 0;
+    st->status = !ok ? FA_ERR_DEVICE : !regs_ok ? FA_ERR_BUILD : FA_OK;
   });
-  return st->ok ? st : nullptr;
+  if (st->status != FA_OK) {
+    if (why) *why = st->status;
+    return nullptr;
+  }
+  return st;
 }
+
+// device_state() for an entry point: the state, or the status to return.
+#define FA_DEVICE_OR_RETURN(var)              \
+  int var##_why = FA_ERR_DEVICE;              \
+  DeviceState* var = device_state(&var##_why); \
+  if (!var) return var##_why
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -163,17 +176,17 @@ constexpr CUtensorMapDataType map_type() {
 int check_heads(int H, int Hkv) { return (Hkv >= 1 && Hkv <= H && H % Hkv == 0) ? FA_OK : FA_ERR_SHAPE; }
 
 template <typename E>
-int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties, int B, int H,
-               int Hkv, int N, int d, int causal, float scale, int fix_mode, cudaStream_t stream) {
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties, int32_t* one_hit,
+               float* o_f32, int B, int H, int Hkv, int N, int d, int causal, float scale, int fix_mode,
+               cudaStream_t stream) {
   constexpr bool kF16 = E::kMmaFmt == 0;
   if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
   int rc = check_common(B, H, N, d, causal, scale);
   if (rc != FA_OK) return rc;
   if ((rc = check_heads(H, Hkv)) != FA_OK) return rc;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGN;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(o_f32)) return FA_ERR_ALIGN;
   if (fix_mode < 0 || fix_mode > 5) return FA_ERR_FIXMODE;
-  DeviceState* st = device_state();
-  if (!st) return FA_ERR_DEVICE;
+  FA_DEVICE_OR_RETURN(st);
   const int BH = B * H;
   CUtensorMap mq, mk, mv;
   constexpr CUtensorMapDataType dt = map_type<E>();
@@ -186,6 +199,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.ties = ties;
+  prm.one_hit = one_hit;
+  prm.o_f32 = o_f32;
   prm.dev_error = st->dev_error;
   prm.BH = BH;
   prm.N = N;
@@ -225,27 +240,8 @@ extern "C" {
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            int causal, float scale, int fix_mode, void* stream) {
-  return launch_fwd<ElemBF16>(q, k, v, o, lse, nullptr, B, H, H, N, d, causal, scale, fix_mode,
+  return launch_fwd<ElemBF16>(q, k, v, o, lse, nullptr, nullptr, nullptr, B, H, H, N, d, causal, scale, fix_mode,
                               static_cast<cudaStream_t>(stream));
-}
-
-int fa_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-               int causal, float scale, int fix_mode, void* stream) {
-  return launch_fwd<ElemF16>(q, k, v, o, lse, nullptr, B, H, H, N, d, causal, scale, fix_mode,
-                             static_cast<cudaStream_t>(stream));
-}
-
-int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
-               int d, int causal, float scale, int fix_mode, void* stream) {
-  return launch_fwd<ElemBF16>(q, k, v, o, lse, nullptr, B, H, Hkv, N, d, causal, scale, fix_mode,
-                    static_cast<cudaStream_t>(stream));
-}
-
-int fa_fwd_ties(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties, int B, int H,
-                int N, int d, int causal, float scale, int fix_mode, void* stream) {
-  if (!ties) return FA_ERR_NULL;
-  return launch_fwd<ElemBF16>(q, k, v, o, lse, ties, B, H, H, N, d, causal, scale, fix_mode,
-                    static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -269,7 +265,8 @@ int pre_impl(const void* o, const void* dout, void* workspace, size_t workspace_
   if (!aligned16(o) || !aligned16(dout)) return FA_ERR_ALIGN;
   if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, N, d))
     return FA_ERR_WORKSPACE;
-  if (!device_state()) return FA_ERR_DEVICE;
+  FA_DEVICE_OR_RETURN(st);
+  (void)st;
   const size_t rows = size_t(B) * H * N;
   float* dq_acc = static_cast<float*>(workspace);
   float* dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256(rows * d * sizeof(float)));
@@ -295,8 +292,7 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse,
     return FA_ERR_ALIGN;
   if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, N, d))
     return FA_ERR_WORKSPACE;
-  DeviceState* st = device_state();
-  if (!st) return FA_ERR_DEVICE;
+  FA_DEVICE_OR_RETURN(st);
   const int BH = B * H;
   const size_t rows = size_t(BH) * N;
   const int BHkv = B * Hkv;
@@ -340,7 +336,8 @@ int finish_impl(void* dq, const void* workspace, size_t workspace_bytes, int B, 
   if (!aligned16(dq)) return FA_ERR_ALIGN;
   if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, N, d))
     return FA_ERR_WORKSPACE;
-  if (!device_state()) return FA_ERR_DEVICE;
+  FA_DEVICE_OR_RETURN(st);
+  (void)st;
   const long long n8 = (long long)B * H * N * d / 8;
   const int threads = 256;
   const cudaError_t e = launch(fa_bwd_dq_kernel<E>, dim3(unsigned((n8 + threads - 1) / threads)), dim3(threads), 0,
@@ -363,7 +360,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     return FA_ERR_ALIGN;
   if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, N, d))
     return FA_ERR_WORKSPACE;
-  if (!device_state()) return FA_ERR_DEVICE;
+  FA_DEVICE_OR_RETURN(st);
+  (void)st;
   rc = pre_impl<E>(o, dout, workspace, workspace_bytes, B, H, N, d, stream);
   if (rc != FA_OK) return rc;
   rc = bwd_main_impl<E>(q, k, v, lse, dout, dk, dv, workspace, workspace_bytes, B, H, Hkv, N, d, causal, scale,
@@ -394,13 +392,6 @@ int fa_bwd_finish(void* dq, const void* workspace, size_t workspace_bytes, int B
   return finish_impl<ElemBF16>(dq, workspace, workspace_bytes, B, H, N, d, scale, stream);
 }
 
-int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
-               void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N,
-               int d, int causal, float scale, void* stream) {
-  return bwd_impl<ElemBF16>(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, N, d, causal,
-                            scale, stream);
-}
-
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
            void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
            int causal, float scale, void* stream) {
@@ -408,21 +399,30 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
                             scale, stream);
 }
 
-int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
-               void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
-               int causal, float scale, void* stream) {
-  return bwd_impl<ElemF16>(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, H, N, d, causal,
-                           scale, stream);
-}
-
-int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties, int B, int H,
-              int Hkv, int N, int d, int causal, float scale, int fix_mode, int elem, void* stream) {
+// The general forward for element format `elem`, with the optional records.
+static int fwd_elem(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties,
+                    int32_t* one_hit, float* o_f32, int B, int H, int Hkv, int N, int d, int causal, float scale,
+                    int fix_mode, int elem, void* stream) {
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (elem == FA_ELEM_BF16)
-    return launch_fwd<ElemBF16>(q, k, v, o, lse, ties, B, H, Hkv, N, d, causal, scale, fix_mode, s);
+    return launch_fwd<ElemBF16>(q, k, v, o, lse, ties, one_hit, o_f32, B, H, Hkv, N, d, causal, scale, fix_mode, s);
   if (elem == FA_ELEM_F16)
-    return launch_fwd<ElemF16>(q, k, v, o, lse, ties, B, H, Hkv, N, d, causal, scale, fix_mode, s);
+    return launch_fwd<ElemF16>(q, k, v, o, lse, ties, one_hit, o_f32, B, H, Hkv, N, d, causal, scale, fix_mode, s);
   return FA_ERR_ARG;
+}
+
+int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
+              int d, int causal, float scale, int fix_mode, int elem, void* stream) {
+  return fwd_elem(q, k, v, o, lse, nullptr, nullptr, nullptr, B, H, Hkv, N, d, causal, scale, fix_mode, elem,
+                  stream);
+}
+
+int fa_fwd_debug(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* tie_count_out,
+                 int32_t* one_hit_out, float* o_f32_out, int B, int H, int Hkv, int N, int d, int causal,
+                 float scale, int fix_mode, int elem, void* stream) {
+  if (!tie_count_out && !one_hit_out && !o_f32_out) return FA_ERR_NULL;
+  return fwd_elem(q, k, v, o, lse, tie_count_out, one_hit_out, o_f32_out, B, H, Hkv, N, d, causal, scale, fix_mode,
+                  elem, stream);
 }
 
 int fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
@@ -452,6 +452,9 @@ const char* fa_status_string(int status) {
       return "an argument is out of range: causal not 0 or 1, scale not finite and > 0, elem not an fa_elem "
              "value, or a watchdog timeout outside 1..1000000 us";
     case FA_ERR_DEVICE: return "no sm_100 device, or tensor-map encoding unavailable";
+    case FA_ERR_BUILD:
+      return "the library was compiled with a register count per thread that its kernels' register split "
+             "does not expect (rebuild with the flags in build.py)";
     case FA_ERR_SCRATCH_LIMIT:
       return "fa_bwd_noalloc: fa_bwd_workspace_size() exceeds FA_BWD_NOALLOC_SCRATCH_BYTES (32 MiB)";
     default: return "unknown status";
@@ -460,16 +463,14 @@ const char* fa_status_string(int status) {
 
 int fa_watchdog_selftest(unsigned timeout_us, void* stream) {
   if (timeout_us < 1 || timeout_us > 1000000) return FA_ERR_ARG;
-  DeviceState* st = device_state();
-  if (!st) return FA_ERR_DEVICE;
+  FA_DEVICE_OR_RETURN(st);
   const cudaError_t e = launch(fa_watchdog_selftest_kernel, dim3(1), dim3(64), 0, static_cast<cudaStream_t>(stream),
                                st->dev_error, uint64_t(timeout_us) * 1000ull);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 int fa_check_device_error(void* stream) {
-  DeviceState* st = device_state();
-  if (!st) return FA_ERR_DEVICE;
+  FA_DEVICE_OR_RETURN(st);
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
   int flag = 0;
   if (cudaMemcpy(&flag, st->dev_error, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_LAUNCH;
@@ -531,7 +532,8 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
       !aligned16(dk) || !aligned16(dv))
     return FA_ERR_ALIGN;
   if (fa_bwd_workspace_size(B, H, N, d) > FA_BWD_NOALLOC_SCRATCH_BYTES) return FA_ERR_SCRATCH_LIMIT;
-  if (!device_state()) return FA_ERR_DEVICE;
+  FA_DEVICE_OR_RETURN(st);
+  (void)st;
   void* scratch = bwd_scratch();
   if (!scratch) return FA_ERR_DEVICE;
   // fa_bwd's first launch zeroes the accumulator and rewrites D, so what the

@@ -33,7 +33,9 @@ namespace fa {
 struct FwdParams {
   void* o;              // [BH, N, D] of the element type
   float* lse;           // [BH, N]
-  int32_t* ties;        // [BH, N] or nullptr
+  int32_t* ties;        // [BH, N] or nullptr: the detector record
+  int32_t* one_hit;     // [BH, N] or nullptr: entries with P_bar == 1.0 under the final shift
+  float* o_f32;         // [BH, N, D] or nullptr: O before its rounding to the element format
   int* dev_error;       // library error flag
   int BH, N, n_pairs, causal;   // BH = batch * query heads
   int H, group;         // query heads per batch entry; query heads per K/V head (1 = no sharing)
@@ -344,6 +346,7 @@ __global__ void __launch_bounds__(384, 1)
       bool ever_repeated = false;   // the running max occurred >= 2 times at some tile
       float l_bar = 0.f;    // running sum of the rounded P_bar (self-normalised mode only)
       int cnt_near = 0;     // entries whose P rounds to 1 under the current shift (near-tie mode)
+      int hits = 0;         // entries packed as P_bar == 1.0 since the shift last moved (one_hit record)
 
       for (int j = 0; j < n_t; ++j) {
         const uint32_t ph = (it_cnt + j) & 1;
@@ -456,11 +459,21 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
         }
         float rs_bar = 0.f;
+        // one_hit record: a move of the shift rescales everything packed so
+        // far by alpha != 1, so only entries packed under the final shift
+        // enter O with weight P_bar; count those that are exactly 1.0
+        const bool moved = (ms_new != ms) || (raise != raised);
+        int th = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = E::pack(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]);
+          if (p.one_hit) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              th += int((pk[i] & 0xffffu) == E::kOneBits) + int((pk[i] >> 16) == E::kOneBits);
+          }
           if (kVariants && p.self_norm) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -471,6 +484,7 @@ __global__ void __launch_bounds__(384, 1)
           tmem_st16(t_p + c * 16, pk);
         }
         l_bar = l_bar * alpha + rs_bar;
+        hits = (moved ? 0 : hits) + th;
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
           const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll 1
@@ -511,8 +525,14 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld_wait(o);
         const float inv_l = 1.f / ((kVariants && p.self_norm) ? l_bar : l);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          ow[c * 16 + i] = E::pack(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * inv_l);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) ow[c * 16 + i] = E::pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1]));
+        if (p.o_f32 && row < p.N) {   // the values whose rounding O is
+          uint4* dst = reinterpret_cast<uint4*>(p.o_f32 + (size_t(w.bh) * p.N + row) * D + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        }
       }
       // O_t is in registers: the next item's first P_bar V may overwrite it
       tc_fence_before();
@@ -522,7 +542,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(ow[4 * i], ow[4 * i + 1], ow[4 * i + 2], ow[4 * i + 3]);
         p.lse[size_t(w.bh) * p.N + row] = (ms + (raised ? p.delta_log2 : 0.f) + lg2(l)) * kLn2;
-        if (p.ties) p.ties[size_t(w.bh) * p.N + row] = cnt | (ever_repeated ? (1 << 30) : 0);
+        if (p.ties)
+          p.ties[size_t(w.bh) * p.N + row] = cnt | (raised ? (1 << 29) : 0) | (ever_repeated ? (1 << 30) : 0);
+        if (p.one_hit) p.one_hit[size_t(w.bh) * p.N + row] = hits;
       }
       it_cnt += n_t;
     }

@@ -456,6 +456,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 struct ElemBF16 {
   using T = __nv_bfloat16;
   static constexpr uint32_t kMmaFmt = 1;
+  static constexpr uint32_t kOneBits = 0x3F80u;   // 1.0
   static __device__ __forceinline__ uint32_t pack(float lo, float hi) { return pack_bf16(lo, hi); }
   static __device__ __forceinline__ float2 unpack(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
@@ -465,6 +466,7 @@ struct ElemBF16 {
 struct ElemF16 {
   using T = __half;
   static constexpr uint32_t kMmaFmt = 0;
+  static constexpr uint32_t kOneBits = 0x3C00u;   // 1.0
   static __device__ __forceinline__ uint32_t pack(float lo, float hi) { return pack_f16(lo, hi); }
   static __device__ __forceinline__ float2 unpack(uint32_t w) {
     return __half22float2(*reinterpret_cast<const __half2*>(&w));

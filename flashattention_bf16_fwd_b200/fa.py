@@ -13,21 +13,21 @@ import os
 import torch
 
 __all__ = [
-    "FAError", "LIB_PATH", "lib", "fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_fwd_f16", "fa_bwd", "fa_bwd_gqa",
-    "fa_bwd_f16", "fa_fwd_ex", "fa_bwd_ex", "FA_ELEM_BF16", "FA_ELEM_F16", "fa_bwd_workspace_size",
-    "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc", "fa_watchdog_selftest",
-    "fa_status_string", "fa_check_device_error", "EXPORTED", "attention_fwd", "attention_bwd",
+    "FAError", "LIB_PATH", "lib", "fa_fwd", "fa_bwd", "fa_fwd_ex", "fa_bwd_ex", "fa_fwd_debug", "FA_ELEM_BF16",
+    "FA_ELEM_F16", "fa_bwd_workspace_size", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc",
+    "fa_watchdog_selftest", "fa_status_string", "fa_check_device_error", "EXPORTED", "attention_fwd",
+    "attention_bwd", "TIE_COUNT_MASK", "TIE_RAISED_BIT", "TIE_FIRED_BIT",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
 
 FA_OK = 0
 FA_ELEM_BF16, FA_ELEM_F16 = 0, 1
-EXPORTED = ("fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_f16", "fa_bwd_f16", "fa_fwd_ex", "fa_bwd_ex",
-            "fa_bwd_workspace_size",
-            "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
-            "fa_bwd_finish", "fa_bwd_noalloc", "fa_watchdog_selftest", "fa_status_string",
-            "fa_check_device_error")
+# fa_fwd_debug's tie record: the count, the final shift raised, the detector fired
+TIE_COUNT_MASK, TIE_RAISED_BIT, TIE_FIRED_BIT = (1 << 29) - 1, 1 << 29, 1 << 30
+EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_bwd_ex", "fa_fwd_debug", "fa_bwd_workspace_size", "fa_bwd",
+            "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc", "fa_watchdog_selftest",
+            "fa_status_string", "fa_check_device_error")
 
 
 class FAError(RuntimeError):
@@ -45,20 +45,12 @@ def _load() -> ctypes.CDLL:
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     so.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     so.fa_fwd.restype = i
-    so.fa_fwd_ties.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
-    so.fa_fwd_ties.restype = i
-    so.fa_fwd_f16.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
-    so.fa_fwd_f16.restype = i
-    so.fa_bwd_f16.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, vp]
-    so.fa_bwd_f16.restype = i
-    so.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
-    so.fa_fwd_gqa.restype = i
-    so.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, f, vp]
-    so.fa_bwd_gqa.restype = i
-    so.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+    so.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
     so.fa_fwd_ex.restype = i
     so.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, f, i, vp]
     so.fa_bwd_ex.restype = i
+    so.fa_fwd_debug.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+    so.fa_fwd_debug.restype = i
     so.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     so.fa_bwd_workspace_size.restype = sz
     so.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, vp]
@@ -117,40 +109,6 @@ def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, fix_mode: int, stream=No
                       int(fix_mode), _stream(stream))
 
 
-def fa_fwd_ties(q, k, v, o, lse, ties, causal: bool, scale: float, fix_mode: int, stream=None) -> int:
-    B, H, N, d = _shape(q)
-    return lib.fa_fwd_ties(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(ties), B, H, N, d, int(causal),
-                           float(scale), int(fix_mode), _stream(stream))
-
-
-def fa_fwd_f16(q, k, v, o, lse, causal: bool, scale: float, fix_mode: int, stream=None) -> int:
-    B, H, N, d = _shape(q)
-    return lib.fa_fwd_f16(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, int(causal), float(scale),
-                          int(fix_mode), _stream(stream))
-
-
-def fa_bwd_f16(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool, scale: float, stream=None) -> int:
-    B, H, N, d = _shape(q)
-    return lib.fa_bwd_f16(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
-                          _ptr(workspace), _nbytes(workspace), B, H, N, d, int(causal), float(scale),
-                          _stream(stream))
-
-
-def fa_fwd_gqa(q, k, v, o, lse, causal: bool, scale: float, fix_mode: int, stream=None) -> int:
-    B, H, N, d = _shape(q)
-    Hkv = k.shape[1]
-    return lib.fa_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, N, d, int(causal), float(scale),
-                          int(fix_mode), _stream(stream))
-
-
-def fa_bwd_gqa(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool, scale: float, stream=None) -> int:
-    B, H, N, d = _shape(q)
-    Hkv = k.shape[1]
-    return lib.fa_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
-                          _ptr(workspace), _nbytes(workspace), B, H, Hkv, N, d, int(causal), float(scale),
-                          _stream(stream))
-
-
 def _elem(t) -> int:
     if t.dtype == torch.bfloat16:
         return FA_ELEM_BF16
@@ -159,11 +117,21 @@ def _elem(t) -> int:
     raise ValueError(f"tensors must be bfloat16 or float16, not {t.dtype}")
 
 
-def fa_fwd_ex(q, k, v, o, lse, ties, causal: bool, scale: float, fix_mode: int, stream=None) -> int:
-    """The general forward: element format from q's dtype, Hkv from k's head count, ties optional."""
+def fa_fwd_ex(q, k, v, o, lse, causal: bool, scale: float, fix_mode: int, stream=None) -> int:
+    """The general forward: element format from q's dtype, Hkv from k's head count."""
     B, H, N, d = _shape(q)
-    return lib.fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(ties), B, H, int(k.shape[1]), N, d,
-                         int(causal), float(scale), int(fix_mode), _elem(q), _stream(stream))
+    return lib.fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, int(k.shape[1]), N, d, int(causal),
+                         float(scale), int(fix_mode), _elem(q), _stream(stream))
+
+
+def fa_fwd_debug(q, k, v, o, lse, ties, one_hit, o_f32, causal: bool, scale: float, fix_mode: int,
+                 stream=None) -> int:
+    """fa_fwd_ex plus the per-row tie record, the P_bar == 1 count and O before
+    its final rounding (each may be None, not all)."""
+    B, H, N, d = _shape(q)
+    return lib.fa_fwd_debug(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(ties), _ptr(one_hit), _ptr(o_f32),
+                            B, H, int(k.shape[1]), N, d, int(causal), float(scale), int(fix_mode), _elem(q),
+                            _stream(stream))
 
 
 def fa_bwd_ex(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool, scale: float, stream=None) -> int:
@@ -244,18 +212,25 @@ def _validate(q, k, v, like_q=()):
 
 
 def attention_fwd(q, k, v, causal: bool = True, scale: float | None = None, fix_mode: int = 1,
-                  stream=None, ties: bool = False):
-    """Allocate O and LSE (and optionally the per-row tie record) and run the
-    forward.  bf16 or fp16 tensors (from q's dtype); k and v may have fewer
-    heads than q (grouped-query attention)."""
+                  stream=None, ties: bool = False, one_hit: bool = False, o_f32: bool = False):
+    """Allocate O and LSE and run the forward; returns (o, lse), followed, in
+    this order and only when asked for, by the per-row tie record (``ties``),
+    the P_bar == 1 count (``one_hit``) and O before its final rounding
+    (``o_f32``), all from fa_fwd_debug.  bf16 or fp16 tensors (from q's dtype);
+    k and v may have fewer heads than q (grouped-query attention)."""
     _validate(q, k, v)
     B, H, N, d = _shape(q)
     scale = d ** -0.5 if scale is None else scale
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     t = torch.empty((B, H, N), dtype=torch.int32, device=q.device) if ties else None
-    _check("fa_fwd_ex", fa_fwd_ex(q, k, v, o, lse, t, causal, scale, fix_mode, stream))
-    return (o, lse, t) if ties else (o, lse)
+    h = torch.empty((B, H, N), dtype=torch.int32, device=q.device) if one_hit else None
+    of = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device) if o_f32 else None
+    if ties or one_hit or o_f32:
+        _check("fa_fwd_debug", fa_fwd_debug(q, k, v, o, lse, t, h, of, causal, scale, fix_mode, stream))
+    else:
+        _check("fa_fwd_ex", fa_fwd_ex(q, k, v, o, lse, causal, scale, fix_mode, stream))
+    return (o, lse) + tuple(x for x, want in ((t, ties), (h, one_hit), (of, o_f32)) if want)
 
 
 def attention_bwd(q, k, v, o, lse, do, causal: bool = True, scale: float | None = None, stream=None,

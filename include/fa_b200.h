@@ -66,8 +66,11 @@ typedef enum {
                             elem not an fa_elem value                         */
   FA_ERR_DEVICE = -10,   /* no sm_100 device, or the driver entry point for
                             tensor maps is unavailable                        */
-  FA_ERR_SCRATCH_LIMIT = -11 /* fa_bwd_noalloc: the problem needs more scratch
+  FA_ERR_SCRATCH_LIMIT = -11, /* fa_bwd_noalloc: the problem needs more scratch
                             than FA_BWD_NOALLOC_SCRATCH_BYTES                 */
+  FA_ERR_BUILD = -12     /* the kernels were compiled with a register count
+                            per thread that their register split does not
+                            expect; nothing is launched                       */
 } fa_status;
 
 /*
@@ -98,77 +101,74 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* l
            int B, int H, int N, int d, int causal, float scale, int fix_mode,
            void* stream);
 
-/*
- * fa_fwd_ties - fa_fwd plus a per-row record of the repeated-max detector:
- *   ties out: int32 [B,H,N], device.  Bits 0-29: the number of visible keys
- *             whose FP32 score equals the row maximum of S (>= 2 means the
- *             fix applies to the final shift when fix_mode is 1, 2 or 3).
- *             Bit 30: set if the detector fired at some key tile: the
- *             running maximum was repeated (fix_mode 0-4), or two or more
- *             entries rounded to 1 (fix_mode 5); with fix_mode 1, 2, 3 or 5
- *             the shift was raised then.  Same kernel as fa_fwd; the extra
- *             store is one int per row.
- */
-FA_API int fa_fwd_ties(const void* q, const void* k, const void* v, void* o, float* lse,
-                int32_t* ties, int B, int H, int N, int d, int causal,
-                float scale, int fix_mode, void* stream);
-
-/*
- * FP16 variant: Q, K, V, O, dO, dQ, dK, dV are fp16 [B,H,N,d] instead of bf16
- * (the pages treat FP16 and BF16 together as the low-precision formats of the
- * instability).  P_bar is rounded to fp16.  The fix modes carry over with the
- * fp16 grid: 1 and 5 map repeated maxima to 1 - 2^-11, the largest fp16 value
- * below 1; 2, 3 and 4 are as in fa_fwd; 5 counts entries whose P rounds to
- * fp16 1.0, i.e. P >= 1 - 2^-12.  Arguments, layouts and the workspace are as
- * in fa_fwd / fa_bwd.
- */
-FA_API int fa_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse,
-                      int B, int H, int N, int d, int causal, float scale, int fix_mode,
-                      void* stream);
-FA_API int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o,
-                      const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                      void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
-                      int causal, float scale, void* stream);
-
-/*
- * Grouped-query attention (GQA; MQA when Hkv == 1), the head layout of the
- * larger Llama 2 models the chibakuma.com page names: H query heads share Hkv
- * key/value heads, query head h reading key/value head h / (H / Hkv).
- *   q, o, dout, dq : bf16 [B,H,N,d];  k, v, dk, dv : bf16 [B,Hkv,N,d];
- *   lse            : float32 [B,H,N].
- * dK and dV of a shared head are the sums over the query heads of its group.
- * Hkv must divide H (FA_ERR_SHAPE otherwise).  Everything else is as in
- * fa_fwd / fa_bwd, which are the Hkv == H case; the workspace is
- * fa_bwd_workspace_size(B, H, N, d) (query heads).
- */
-FA_API int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
-                      int B, int H, int Hkv, int N, int d, int causal, float scale,
-                      int fix_mode, void* stream);
-FA_API int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
-                      const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                      void* workspace, size_t workspace_bytes, int B, int H, int Hkv,
-                      int N, int d, int causal, float scale, void* stream);
-
-/* Element formats of fa_fwd_ex / fa_bwd_ex. */
+/* Element formats of fa_fwd_ex / fa_bwd_ex / fa_fwd_debug. */
 typedef enum { FA_ELEM_BF16 = 0, FA_ELEM_F16 = 1 } fa_elem;
 
 /*
- * fa_fwd_ex / fa_bwd_ex - one call for every combination of the above: the
- * element format `elem` (FA_ELEM_BF16 or FA_ELEM_F16) of every [.,.,N,d]
- * tensor and of P_bar, H query heads over Hkv key/value heads (Hkv == H:
- * ordinary attention), any fix_mode 0-5, and the optional `ties` record of
- * fa_fwd_ties (NULL to skip it).  fa_fwd, fa_fwd_ties, fa_fwd_f16, fa_fwd_gqa
- * and the matching backward calls are this call with their fixed arguments.
+ * fa_fwd_ex / fa_bwd_ex - fa_fwd / fa_bwd for every combination of:
+ *   - elem: the element format (FA_ELEM_BF16 or FA_ELEM_F16) of every
+ *     [.,.,N,d] tensor and of P_bar.  The pages treat FP16 and BF16 together
+ *     as the low-precision formats of the instability (yicaiai article,
+ *     abstract).  With FP16 the fix modes carry over on the fp16 grid: 1 and 5
+ *     map repeated maxima to 1 - 2^-11, the largest fp16 value below 1;
+ *     2, 3 and 4 are as in fa_fwd; 5 counts entries whose P rounds to fp16
+ *     1.0, i.e. P >= 1 - 2^-12.
+ *   - H query heads over Hkv key/value heads (grouped-query attention, the
+ *     head layout of the larger Llama 2 models that "Is Flash Attention
+ *     Stable?" names; MQA when Hkv == 1; ordinary attention when Hkv == H):
+ *     query head h reads key/value head h / (H / Hkv).
+ *       q, o, dout, dq : [B,H,N,d];  k, v, dk, dv : [B,Hkv,N,d];
+ *       lse            : float32 [B,H,N].
+ *     dK and dV of a shared head are the sums over the query heads of its
+ *     group.  Hkv must divide H (FA_ERR_SHAPE otherwise).  The workspace is
+ *     fa_bwd_workspace_size(B, H, N, d) (query heads).
+ *   - any fix_mode 0-5.
+ * fa_fwd and fa_bwd are these calls with elem = FA_ELEM_BF16 and Hkv = H.
  * Layouts, ownership, the workspace and the error codes are theirs;
  * FA_ERR_ARG also reports an unknown elem.
  */
 FA_API int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
-                     int32_t* ties, int B, int H, int Hkv, int N, int d, int causal,
-                     float scale, int fix_mode, int elem, void* stream);
+                     int B, int H, int Hkv, int N, int d, int causal, float scale,
+                     int fix_mode, int elem, void* stream);
 FA_API int fa_bwd_ex(const void* q, const void* k, const void* v, const void* o,
                      const float* lse, const void* dout, void* dq, void* dk, void* dv,
                      void* workspace, size_t workspace_bytes, int B, int H, int Hkv,
                      int N, int d, int causal, float scale, int elem, void* stream);
+
+/*
+ * fa_fwd_debug - fa_fwd_ex plus per-row records that show the fix at work
+ * inside the kernel ("Why Low-Precision Transformer Training Fails",
+ * admirer.cn summary, mechanism 2: detect a repeated row maximum of S and
+ * raise the shift so that every exponent, the maxima included, is strictly
+ * below 1; the same section places the bias in the forward's unnormalised
+ * output).  Same kernel and arithmetic as fa_fwd_ex; O and LSE are
+ * bit-identical to its outputs.  Any of the three records may be NULL, not
+ * all (FA_ERR_NULL).
+ *   tie_count_out out: int32 [B,H,N], device.
+ *       Bits 0-28: the number of visible keys whose FP32 score equals the row
+ *       maximum of S (at most N < 2^25).
+ *       Bit 29: the row's final shift is the raised one, i.e. the fix applies
+ *       to its output (fix_mode 1, 2, 3 with a repeated maximum; fix_mode 5
+ *       with two or more entries that round to 1).
+ *       Bit 30: the detector fired at some key tile: the running maximum was
+ *       repeated (fix_mode 0-4), or two or more entries rounded to 1
+ *       (fix_mode 5).
+ *   one_hit_out   out: int32 [B,H,N], device.  The number of entries of the
+ *       row whose P_bar, as the kernel rounded it for the P_bar V product,
+ *       is exactly 1.0, counted among the entries produced under the row's
+ *       final shift (a move of the shift rescales O and l exactly, so
+ *       entries rounded earlier no longer enter O with weight P_bar).  A row
+ *       whose final shift is raised (bit 29 above) has 0: no exponent reaches
+ *       1.  A row with the plain shift has at least 1 (its maximum).
+ *   o_f32_out     out: float32 [B,H,N,d], device, 16-byte aligned.  O before
+ *       its rounding to the element format: the FP32 values (P_bar V) / l
+ *       whose round-to-nearest-even is the returned O.  It shows the error
+ *       of the P_bar V path without the error of the output's own rounding.
+ */
+FA_API int fa_fwd_debug(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int32_t* tie_count_out, int32_t* one_hit_out, float* o_f32_out,
+                        int B, int H, int Hkv, int N, int d, int causal, float scale,
+                        int fix_mode, int elem, void* stream);
 
 /*
  * fa_bwd_workspace_size - bytes of device scratch fa_bwd needs:

@@ -43,16 +43,21 @@ int main(void) {
   CHECK(fa_fwd(A, A, A, A, L, 1, 1, 128, 64, 2, 0.125f, 1, NULL), FA_ERR_ARG);
   CHECK(fa_fwd(A, A, A, MIS, L, 1, 1, 128, 64, 1, 0.125f, 1, NULL), FA_ERR_ALIGN);
   CHECK(fa_fwd(A, A, A, A, L, 1, 1, 128, 64, 1, 0.125f, 7, NULL), FA_ERR_FIXMODE);
-  CHECK(fa_fwd_ties(A, A, A, A, L, NULL, 1, 1, 128, 64, 1, 0.125f, 1, NULL), FA_ERR_NULL);
-  CHECK(fa_fwd_f16(A, A, A, A, L, 1, 1, 128, 64, 1, 0.125f, 6, NULL), FA_ERR_FIXMODE);
-  CHECK(fa_fwd_gqa(A, A, A, A, L, 1, 4, 3, 128, 64, 1, 0.125f, 1, NULL), FA_ERR_SHAPE);
-  CHECK(fa_fwd_ex(A, A, A, A, L, NULL, 1, 4, 2, 128, 64, 1, 0.125f, 1, 9, NULL), FA_ERR_ARG);
-  CHECK(fa_fwd_ex(A, A, A, A, L, NULL, 1, 4, 2, 128, 64, 1, 0.125f, 1, FA_ELEM_F16 + 1, NULL), FA_ERR_ARG);
+  CHECK(fa_fwd_debug(A, A, A, A, L, NULL, NULL, NULL, 1, 1, 1, 128, 64, 1, 0.125f, 1, FA_ELEM_BF16, NULL),
+        FA_ERR_NULL);
+  CHECK(fa_fwd_debug(A, A, A, A, L, NULL, (int32_t*)A, NULL, 1, 4, 3, 128, 64, 1, 0.125f, 1, FA_ELEM_F16, NULL),
+        FA_ERR_SHAPE);
+  CHECK(fa_fwd_ex(A, A, A, A, L, 1, 1, 1, 128, 64, 1, 0.125f, 6, FA_ELEM_F16, NULL), FA_ERR_FIXMODE);
+  CHECK(fa_fwd_ex(A, A, A, A, L, 1, 4, 3, 128, 64, 1, 0.125f, 1, FA_ELEM_BF16, NULL), FA_ERR_SHAPE);
+  CHECK(fa_fwd_ex(A, A, A, A, L, 1, 4, 2, 128, 64, 1, 0.125f, 1, 9, NULL), FA_ERR_ARG);
+  CHECK(fa_fwd_ex(A, A, A, A, L, 1, 4, 2, 128, 64, 1, 0.125f, 1, FA_ELEM_F16 + 1, NULL), FA_ERR_ARG);
 
   CHECK(fa_bwd(A, A, A, A, L, A, A, A, A, A, ws - 1, 2, 3, 1000, 64, 1, 0.125f, NULL), FA_ERR_WORKSPACE);
   CHECK(fa_bwd(A, A, A, A, L, A, A, A, A, NULL, ws, 2, 3, 1000, 64, 1, 0.125f, NULL), FA_ERR_WORKSPACE);
-  CHECK(fa_bwd_f16(A, A, A, A, L, A, MIS, A, A, A, ws, 2, 3, 1000, 64, 1, 0.125f, NULL), FA_ERR_ALIGN);
-  CHECK(fa_bwd_gqa(A, A, A, A, L, A, A, A, A, A, ws, 2, 3, 2, 1000, 64, 1, 0.125f, NULL), FA_ERR_SHAPE);
+  CHECK(fa_bwd_ex(A, A, A, A, L, A, MIS, A, A, A, ws, 2, 3, 3, 1000, 64, 1, 0.125f, FA_ELEM_F16, NULL),
+        FA_ERR_ALIGN);
+  CHECK(fa_bwd_ex(A, A, A, A, L, A, A, A, A, A, ws, 2, 3, 2, 1000, 64, 1, 0.125f, FA_ELEM_BF16, NULL),
+        FA_ERR_SHAPE);
   CHECK(fa_bwd_ex(A, A, A, A, L, A, A, A, A, A, ws, 2, 3, 3, 1000, 64, 1, 0.125f, -1, NULL), FA_ERR_ARG);
   CHECK(fa_bwd_preprocess(A, NULL, A, ws, 2, 3, 1000, 64, NULL), FA_ERR_NULL);
   CHECK(fa_bwd_main(A, A, A, L, A, A, A, A, ws, 2, 3, 1000, 64, 1, -1.0f, NULL), FA_ERR_ARG);
@@ -60,7 +65,7 @@ int main(void) {
   CHECK(fa_bwd_noalloc(A, A, A, A, L, A, A, A, A, 1, 1, 129056, 64, 1, 0.125f, NULL), FA_ERR_SCRATCH_LIMIT);
   CHECK(fa_watchdog_selftest(0, NULL), FA_ERR_ARG);
 
-  for (s = FA_ERR_SCRATCH_LIMIT; s <= FA_OK; ++s) {
+  for (s = FA_ERR_BUILD; s <= FA_OK; ++s) {
     const char* msg = fa_status_string(s);
     if (!msg || !strlen(msg) || !strcmp(msg, "unknown status")) {
       printf("FAIL status string for %d\n", s);

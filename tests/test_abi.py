@@ -16,6 +16,7 @@ HEADER = os.path.join(ROOT, "include", "fa_b200.h")
 
 FA_OK, FA_ERR_NULL, FA_ERR_SHAPE, FA_ERR_HEADDIM, FA_ERR_ALIGN = 0, -1, -2, -3, -4
 FA_ERR_FIXMODE, FA_ERR_WORKSPACE, FA_ERR_LAUNCH, FA_ERR_TIMEOUT, FA_ERR_ARG, FA_ERR_DEVICE = -5, -6, -7, -8, -9, -10
+FA_ERR_BUILD = -12
 
 
 @pytest.fixture(scope="module")
@@ -31,9 +32,8 @@ def declared_symbols():
 
 
 def test_header_declares_the_boundary():
-    assert declared_symbols() == sorted(["fa_fwd", "fa_fwd_ties", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_f16", "fa_bwd_f16",
-                                         "fa_fwd_ex", "fa_bwd_ex", "fa_bwd_workspace_size", "fa_bwd",
-                                         "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish",
+    assert declared_symbols() == sorted(["fa_fwd", "fa_fwd_ex", "fa_bwd_ex", "fa_fwd_debug", "fa_bwd_workspace_size",
+                                         "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finish",
                                          "fa_bwd_noalloc", "fa_watchdog_selftest", "fa_status_string",
                                          "fa_check_device_error"])
 
@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(fa):
 
 
 def test_status_strings(fa):
-    for code in range(0, -12, -1):
+    for code in range(0, -13, -1):
         s = fa.fa_status_string(code)
         assert s and s != "unknown status"
     assert fa.fa_status_string(-99) == "unknown status"
@@ -91,7 +91,12 @@ def test_fwd_argument_errors(fa):
     assert fwd(fa, o=MIS) == FA_ERR_ALIGN
     assert fwd(fa, fix=6) == FA_ERR_FIXMODE
     assert fwd(fa, fix=-1) == FA_ERR_FIXMODE
-    assert fa.lib.fa_fwd_ties(A, A, A, A, A, None, 1, 1, 128, 64, 1, 0.125, 1, None) == FA_ERR_NULL
+    # fa_fwd_debug needs at least one of its two records
+    assert fa.lib.fa_fwd_debug(A, A, A, A, A, None, None, None, 1, 1, 1, 128, 64, 1, 0.125, 1, 0, None) == FA_ERR_NULL
+    assert fa.lib.fa_fwd_debug(A, A, A, A, A, A, None, None, 1, 1, 1, 128, 64, 1, 0.125, 6, 0, None) == FA_ERR_FIXMODE
+    assert fa.lib.fa_fwd_debug(A, A, A, A, A, None, A, None, 1, 4, 3, 128, 64, 1, 0.125, 1, 0, None) == FA_ERR_SHAPE
+    assert fa.lib.fa_fwd_debug(A, A, A, A, A, None, None, MIS, 1, 1, 1, 128, 64, 1, 0.125, 1, 0, None) == FA_ERR_ALIGN
+    assert fa.lib.fa_fwd_debug(A, A, A, A, A, None, A, None, 1, 1, 1, 128, 64, 1, 0.125, 1, 2, None) == FA_ERR_ARG
 
 
 def test_bwd_argument_errors(fa):
@@ -119,7 +124,7 @@ FA_ERR_SCRATCH_LIMIT = -11
 
 def test_general_entry_point_argument_errors(fa):
     fx = lambda **kw: fa.lib.fa_fwd_ex(*[kw.get(n, dflt) for n, dflt in (
-        ("q", A), ("k", A), ("v", A), ("o", A), ("lse", A), ("ties", None), ("B", 1), ("H", 4), ("Hkv", 2),
+        ("q", A), ("k", A), ("v", A), ("o", A), ("lse", A), ("B", 1), ("H", 4), ("Hkv", 2),
         ("N", 128), ("d", 64), ("causal", 1), ("scale", 0.125), ("fix", 1), ("elem", 0), ("stream", None))])
     assert fx(elem=2) == FA_ERR_ARG
     assert fx(elem=-1) == FA_ERR_ARG
@@ -127,6 +132,11 @@ def test_general_entry_point_argument_errors(fa):
     assert fx(Hkv=3) == FA_ERR_SHAPE
     assert fx(v=None) == FA_ERR_NULL
     assert fx(o=MIS, elem=1) == FA_ERR_ALIGN
+    # grouped heads: Hkv must divide H and not exceed it
+    assert fx(Hkv=0) == FA_ERR_SHAPE
+    assert fx(Hkv=8) == FA_ERR_SHAPE
+    assert fx(d=96, elem=1) == FA_ERR_HEADDIM
+    assert fx(lse=None, elem=1) == FA_ERR_NULL
     ws = fa.fa_bwd_workspace_size(1, 4, 128, 64)
     bx = lambda **kw: fa.lib.fa_bwd_ex(*[kw.get(n, dflt) for n, dflt in (
         ("q", A), ("k", A), ("v", A), ("o", A), ("lse", A), ("do", A), ("dq", A), ("dk", A), ("dv", A),
@@ -136,6 +146,10 @@ def test_general_entry_point_argument_errors(fa):
     assert bx(wsz=ws - 1) == FA_ERR_WORKSPACE
     assert bx(Hkv=8) == FA_ERR_SHAPE
     assert bx(d=96) == FA_ERR_HEADDIM
+    assert bx(Hkv=3) == FA_ERR_SHAPE
+    assert bx(dk=MIS) == FA_ERR_ALIGN
+    assert bx(dk=None) == FA_ERR_NULL
+    assert bx(dq=MIS, elem=0) == FA_ERR_ALIGN
 
 
 def test_binding_checks_shapes_and_dtypes(fa):
@@ -148,34 +162,6 @@ def test_binding_checks_shapes_and_dtypes(fa):
         fa.attention_fwd(q.transpose(2, 3).contiguous().transpose(2, 3), q, q)
     with pytest.raises(ValueError):                   # float32 is not a supported format
         fa.attention_fwd(q.float(), q.float(), q.float())
-
-
-def test_f16_argument_errors(fa):
-    # the fp16 path carries every fix_mode, 0-5
-    assert fa.lib.fa_fwd_f16(A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 6, None) == FA_ERR_FIXMODE
-    assert fa.lib.fa_fwd_f16(A, A, A, A, None, 1, 1, 128, 64, 1, 0.125, 1, None) == FA_ERR_NULL
-    assert fa.lib.fa_fwd_f16(A, A, A, A, A, 1, 1, 128, 96, 1, 0.125, 1, None) == FA_ERR_HEADDIM
-    ws = fa.fa_bwd_workspace_size(1, 1, 128, 64)
-    assert fa.lib.fa_bwd_f16(A, A, A, A, A, A, MIS, A, A, A, ws, 1, 1, 128, 64, 1, 0.125, None) == FA_ERR_ALIGN
-    assert fa.lib.fa_bwd_f16(A, A, A, A, A, A, A, A, A, A, ws - 1, 1, 1, 128, 64, 1, 0.125, None) == FA_ERR_WORKSPACE
-
-
-def test_gqa_argument_errors(fa):
-    def fg(H=4, Hkv=2, d=64, q=A):
-        return fa.lib.fa_fwd_gqa(q, A, A, A, A, 1, H, Hkv, 128, d, 1, 0.125, 1, None)
-
-    def bg(H=4, Hkv=2, dk=A):
-        ws = fa.fa_bwd_workspace_size(1, H, 128, 64)
-        return fa.lib.fa_bwd_gqa(A, A, A, A, A, A, A, dk, A, A, ws, 1, H, Hkv, 128, 64, 1, 0.125, None)
-
-    assert fg(Hkv=3) == FA_ERR_SHAPE          # must divide H
-    assert fg(Hkv=0) == FA_ERR_SHAPE
-    assert fg(Hkv=8) == FA_ERR_SHAPE          # more K/V heads than query heads
-    assert fg(d=96) == FA_ERR_HEADDIM
-    assert fg(q=None) == FA_ERR_NULL
-    assert bg(Hkv=3) == FA_ERR_SHAPE
-    assert bg(dk=MIS) == FA_ERR_ALIGN
-    assert bg(dk=None) == FA_ERR_NULL
 
 
 def test_bwd_noalloc_argument_errors(fa):
@@ -202,9 +188,10 @@ def test_valid_call_without_gpu_reports_device_error(fa):
     assert fa.lib.fa_watchdog_selftest(1000, None) == FA_ERR_DEVICE
     # arguments that pass every check; with a GPU these would launch
     assert fwd(fa, H=32767, N=1024, d=64) == FA_ERR_DEVICE            # one head below the 2^31 bound
-    assert fa.lib.fa_fwd_f16(A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 5, None) == FA_ERR_DEVICE
-    assert fa.lib.fa_fwd_ex(A, A, A, A, A, None, 1, 4, 2, 128, 64, 1, 0.125, 1, 0, None) == FA_ERR_DEVICE
-    assert fa.lib.fa_fwd_ex(A, A, A, A, A, None, 1, 4, 2, 128, 64, 1, 0.125, 5, 1, None) == FA_ERR_DEVICE
+    assert fa.lib.fa_fwd_ex(A, A, A, A, A, 1, 1, 1, 128, 64, 1, 0.125, 5, 1, None) == FA_ERR_DEVICE
+    assert fa.lib.fa_fwd_ex(A, A, A, A, A, 1, 4, 2, 128, 64, 1, 0.125, 1, 0, None) == FA_ERR_DEVICE
+    assert fa.lib.fa_fwd_ex(A, A, A, A, A, 1, 4, 2, 128, 64, 1, 0.125, 5, 1, None) == FA_ERR_DEVICE
+    assert fa.lib.fa_fwd_debug(A, A, A, A, A, A, A, A, 1, 4, 2, 128, 64, 1, 0.125, 1, 0, None) == FA_ERR_DEVICE
     ws4 = fa.fa_bwd_workspace_size(1, 4, 128, 64)
     assert fa.lib.fa_bwd_ex(A, A, A, A, A, A, A, A, A, A, ws4, 1, 4, 2, 128, 64, 1, 0.125, 1, None) == FA_ERR_DEVICE
 

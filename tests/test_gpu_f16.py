@@ -1,4 +1,4 @@
-"""The FP16 variant (fa_fwd_f16 / fa_bwd_f16) against the FP64 oracle.
+"""The FP16 variant (fa_fwd_ex / fa_bwd_ex with FP16 tensors) against the FP64 oracle.
 
 Inputs are drawn in float32 and cast once to fp16, so they use fp16's full
 11-bit significand.  The exact oracle and the tolerances of the bf16 parity
@@ -31,13 +31,13 @@ def run(fa, q, k, v, do, causal, scale, fix_mode, bwd=True):
     B, H, N, d = q.shape
     o = torch.empty_like(qd)
     lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
-    assert fa.fa_fwd_f16(qd, kd, vd, o, lse, causal, scale, fix_mode) == 0
+    assert fa.fa_fwd_ex(qd, kd, vd, o, lse, causal, scale, fix_mode) == 0
     out = {"o": o, "lse": lse}
     if bwd:
         dod = do.to(dev)
         dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
         ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
-        assert fa.fa_bwd_f16(qd, kd, vd, o, lse, dod, dq, dk, dv, ws, causal, scale) == 0
+        assert fa.fa_bwd_ex(qd, kd, vd, o, lse, dod, dq, dk, dv, ws, causal, scale) == 0
         out.update(dq=dq, dk=dk, dv=dv)
     torch.cuda.synchronize()
     assert fa.fa_check_device_error() == 0

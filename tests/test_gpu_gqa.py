@@ -44,10 +44,10 @@ def test_gqa_parity(fa, B, H, Hkv, N, d, causal):
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
     o = torch.empty_like(qd)
     lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
-    assert fa.fa_fwd_gqa(qd, kd, vd, o, lse, causal, scale, 1) == 0
+    assert fa.fa_fwd_ex(qd, kd, vd, o, lse, causal, scale, 1) == 0
     dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
     ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
-    assert fa.fa_bwd_gqa(qd, kd, vd, o, lse, dod, dq, dk, dv, ws, causal, scale) == 0
+    assert fa.fa_bwd_ex(qd, kd, vd, o, lse, dod, dq, dk, dv, ws, causal, scale) == 0
     torch.cuda.synchronize()
     assert fa.fa_check_device_error() == 0
 
@@ -64,20 +64,19 @@ def test_gqa_parity(fa, B, H, Hkv, N, d, causal):
 
 
 def test_gqa_with_one_group_per_head_is_plain_attention(fa):
-    """Hkv == H runs the same arithmetic as fa_fwd / fa_bwd, bit for bit (dQ up
-    to the order of its reduce-adds)."""
+    """Hkv == H through fa_fwd_ex / fa_bwd_ex runs the same arithmetic as
+    fa_fwd / fa_bwd, bit for bit (dQ up to the order of its reduce-adds)."""
     B, H, N, d = 1, 3, 333, 64
     q, k, v, do = (t.cuda() for t in draw(B, H, H, N, d, seed=5))
-    o1, l1 = fa.attention_fwd(q, k, v, causal=True, scale=0.125, fix_mode=1)
-    o2 = torch.empty_like(q)
-    l2 = torch.empty_like(l1)
-    assert fa.fa_fwd_gqa(q, k, v, o2, l2, True, 0.125, 1) == 0
+    o1, l1 = torch.empty_like(q), torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+    assert fa.fa_fwd(q, k, v, o1, l1, True, 0.125, 1) == 0
+    o2, l2 = fa.attention_fwd(q, k, v, causal=True, scale=0.125, fix_mode=1)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
-    dq1, dk1, dv1 = fa.attention_bwd(q, k, v, o1, l1, do, causal=True, scale=0.125)
-    dq2, dk2, dv2 = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dq1, dk1, dv1 = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
-    assert fa.fa_bwd_gqa(q, k, v, o1, l1, do, dq2, dk2, dv2, ws, True, 0.125) == 0
+    assert fa.fa_bwd(q, k, v, o1, l1, do, dq1, dk1, dv1, ws, True, 0.125) == 0
+    dq2, dk2, dv2 = fa.attention_bwd(q, k, v, o1, l1, do, causal=True, scale=0.125)
     torch.cuda.synchronize()
     assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
     assert normwise_rel_err(dq1.float().cpu().numpy(), dq2.float().cpu().numpy().astype(np.float64)) < 2.0 ** -8

@@ -10,7 +10,10 @@ depend on the scratch and must match fa_bwd bit for bit.  dQ is summed with
 reduce-adds in an order that varies from run to run, so after its rounding to
 bf16 a few elements land one bf16 step apart; it is held to the gradient
 tolerance of the parity tests (normwise 5e-2).  A d = 128 call follows to
-cover the other kernel instantiation.
+cover the other kernel instantiation.  Last, once every kernel has run (so
+that loading their code has already claimed its memory), a call on a shape
+not seen before must leave the device's free memory exactly where it was:
+the call allocates nothing.
 """
 import pytest
 import torch
@@ -45,3 +48,16 @@ def test_noalloc_matches_fa_bwd_on_calls_in_a_row():
         assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2]), (w, seed)
         err = normwise_rel_err(dq.float().cpu().numpy(), ref[0].float().cpu().numpy())
         assert err <= GRAD_RTOL, (w, seed, err)
+    # a new shape after every kernel has been loaded: no device memory changes hands
+    w = Workload("noalloc", 1, 2, 513, 64, causal=True)
+    x = make_inputs(w, seed=4)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, lse = fa.attention_fwd(q, k, v, causal=w.causal, scale=w.scale, fix_mode=1)
+    got = [torch.empty_like(q) for _ in range(3)]
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    assert fa.fa_bwd_noalloc(q, k, v, o, lse, do, *got, w.causal, w.scale) == 0
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert fa.fa_check_device_error() == 0
+    assert free_after == free_before, (free_before, free_after)
