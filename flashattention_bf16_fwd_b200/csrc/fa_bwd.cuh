@@ -87,6 +87,7 @@ struct BwdParams {
   int* dev_error;
   int BH, N, n_kv, causal;   // BH = batch * K/V heads
   int H, group;         // query heads per batch entry; query heads per K/V head (1 = no sharing)
+  int hg;               // K/V heads per scheduling group (their Q, dO and dQ fit in the L2 together)
   float scale, scale_log2;
 };
 
@@ -137,20 +138,25 @@ struct BwdLayout {
   __host__ __device__ static constexpr uint32_t dst_col(int k) { return kTmDP + 64 * (k >> 2) + 8 * (k & 3); }
 };
 
-// One work item = one (batch*head, 128-key tile); items are numbered heavy
-// first (causal: the first key tiles are seen by the most query tiles).  CTAs
-// are persistent and sweep the sorted items with snake_item()
+// One work item = one (batch*K/V head, 128-key tile).  It loops over the
+// query tiles that see those keys, for each query head of the group that
+// shares the K/V head (dK, dV accumulate over all of them): n_it steps.
+// Items are numbered in groups of hg K/V heads whose Q, dO and dQ accumulator
+// fit in the L2 together; within a group heavy first (causal: the first key
+// tiles are seen by the most query tiles).  CTAs are persistent and sweep the
+// items with snake_item().
 struct BwdItem {
   int bh, kv_tile, key0, i_start, n_it_head, n_it;
 };
 
-// One work item = one (batch*K/V head, 128-key tile).  It loops over the
-// query tiles that see those keys, for each query head of the group that
-// shares the K/V head (dK, dV accumulate over all of them): n_it steps.
 __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
   BwdItem w;
-  w.kv_tile = item / p.BH;
-  w.bh = item % p.BH;
+  const int per_group = p.hg * p.n_kv;
+  const int grp = item / per_group;
+  const int j = item - grp * per_group;
+  const int hg = min(p.hg, p.BH - grp * p.hg);   // the last group may be smaller
+  w.kv_tile = j / hg;
+  w.bh = grp * p.hg + (j - w.kv_tile * hg);
   w.key0 = w.kv_tile * 128;
   const int n_q = (p.N + 127) / 128;
   w.i_start = p.causal ? w.kv_tile : 0;

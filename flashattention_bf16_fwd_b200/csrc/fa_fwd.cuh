@@ -26,6 +26,8 @@
 // and is the A operand of O_t += P_bar V (V is the MN-major B operand).
 #pragma once
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace fa {
@@ -39,6 +41,7 @@ struct FwdParams {
   int* dev_error;       // library error flag
   int BH, N, n_pairs, causal;   // BH = batch * query heads
   int H, group;         // query heads per batch entry; query heads per K/V head (1 = no sharing)
+  int hg;               // heads per scheduling group (their K/V fit in the L2 together)
   float scale_log2;     // scale * log2(e): S -> base-2 exponent domain
   float delta_log2;     // shift added to m on repeated-max rows (0 = fix off)
   float fix_factor;     // 2^-delta_log2: P at a repeated maximum (1 - 2^-8 or, in fp16, 1 - 2^-11; 0.5; exp(-1/16))
@@ -75,16 +78,23 @@ struct FwdLayout {
 };
 
 // One work item = one (batch*head, pair of query tiles).  Items are numbered
-// heavy first (causal: the last query tiles see the most keys); the CTAs are
-// persistent and sweep the sorted items with snake_item()
+// in groups of hg heads whose K/V fit in the L2 together, so that the CTAs in
+// flight stream few heads at once; within a group heavy first (causal: the
+// last query tiles see the most keys).  The CTAs are persistent and sweep the
+// items with snake_item().
 struct FwdItem {
   int bh, q0_row, n0, n1, nmax;
 };
 
 __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
   FwdItem it;
-  const int pair = p.causal ? (p.n_pairs - 1 - item / p.BH) : item / p.BH;
-  it.bh = item % p.BH;
+  const int per_group = p.hg * p.n_pairs;
+  const int grp = item / per_group;
+  const int j = item - grp * per_group;
+  const int hg = min(p.hg, p.BH - grp * p.hg);   // the last group may be smaller
+  const int rank = j / hg;
+  it.bh = grp * p.hg + (j - rank * hg);
+  const int pair = p.causal ? (p.n_pairs - 1 - rank) : rank;
   it.q0_row = pair * 256;
   const int n_kv = (p.N + 127) / 128;
   it.n0 = p.causal ? min(2 * pair + 1, n_kv) : n_kv;
@@ -102,7 +112,9 @@ __device__ __forceinline__ constexpr float rounds_to_one() {
 
 // E: the element format (ElemBF16 or ElemF16) of Q, K, V, O and of P_bar.
 // kVariants: compiled with the code of fix_mode 4 (self-normalised) and 5
-// (near ties); the other instantiation, used for fix_mode 0-3, leaves it out.
+// (near ties) and with the debug records (tie record, P_bar == 1 count, O
+// before rounding); the other instantiation, used for fix_mode 0-3 without
+// records, leaves all of it out.
 template <int D, bool kVariants, typename E = ElemBF16>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -358,6 +370,10 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, r[c]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld_wait(r[c]);
+        if (L::kSepP) {                                // S_t is in registers: the next S may overwrite it
+          tc_fence_before();
+          mbar_arrive(&s_free[t]);
+        }
         float s[128];
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(r[i >> 5][i & 31]);
@@ -424,29 +440,12 @@ __global__ void __launch_bounds__(384, 1)
         const bool raise = p.fix && det >= 2;
         f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), ea, eb);
         float rs = ea + eb;
-        if (__any_sync(0xffffffffu, raise && !raise_early)) {
-          // Rare path: some row of this warp became repeated in this tile.  S is
-          // still intact in TMEM; recompute P for the whole warp (unchanged rows
-          // get the identical arithmetic) and scale the repeated rows by 2^-delta.
-          uint32_t q[4][32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, q[c]);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld_wait(q[c]);
-          float rs_raised = 0.f;
-#pragma unroll
-          for (int i = 0; i < 128; ++i) {
-            const float sv = (masked && key0 + i > limit) ? kNegInf : __uint_as_float(q[i >> 5][i & 31]);
-            const float pv = ex2(fmaf(sv, sl2, -ms_new));
-            s[i] = raise ? pv * kFixFactor : pv;
-            rs_raised += s[i];
-          }
-          if (raise) rs = rs_raised;
-        }
-        if (L::kSepP) {                                // S_t is read: the next S may overwrite it
-          tc_fence_before();
-          mbar_arrive(&s_free[t]);
-        }
+        // Rare path: a row that became repeated in this tile had its P computed
+        // with the plain shift; it is packed scaled by 2^-delta, which is the
+        // raised shift (the scaled pack runs only in warps that need it)
+        const bool rare = __any_sync(0xffffffffu, raise && !raise_early);
+        const float pf = (raise && !raise_early) ? kFixFactor : 1.f;
+        if (raise && !raise_early) rs *= kFixFactor;
         // rescale of the running O and l: exact, whenever the shift moves
         float alpha = ex2(ms - ms_new);
         if (raise != raised) alpha = raise ? alpha * kFixFactor : alpha / kFixFactor;
@@ -464,25 +463,38 @@ __global__ void __launch_bounds__(384, 1)
         // enter O with weight P_bar; count those that are exactly 1.0
         const bool moved = (ms_new != ms) || (raise != raised);
         int th = 0;
+        auto pack_store = [&](auto scaled) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = E::pack(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]);
-          if (p.one_hit) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              th += int((pk[i] & 0xffffu) == E::kOneBits) + int((pk[i] >> 16) == E::kOneBits);
-          }
-          if (kVariants && p.self_norm) {
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float2 pp = E::unpack(pk[i]);
-              rs_bar += pp.x + pp.y;
+              float a = s[c * 32 + 2 * i], b = s[c * 32 + 2 * i + 1];
+              if (decltype(scaled)::value) {
+                a *= pf;
+                b *= pf;
+              }
+              pk[i] = E::pack(a, b);
             }
+            if (kVariants && p.one_hit) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                th += int((pk[i] & 0xffffu) == E::kOneBits) + int((pk[i] >> 16) == E::kOneBits);
+            }
+            if (kVariants && p.self_norm) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float2 pp = E::unpack(pk[i]);
+                rs_bar += pp.x + pp.y;
+              }
+            }
+            tmem_st16(t_p + c * 16, pk);
           }
-          tmem_st16(t_p + c * 16, pk);
-        }
+        };
+        if (rare)
+          pack_store(std::true_type{});
+        else
+          pack_store(std::false_type{});
         l_bar = l_bar * alpha + rs_bar;
         hits = (moved ? 0 : hits) + th;
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -528,7 +540,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * inv_l);
 #pragma unroll
         for (int i = 0; i < 16; ++i) ow[c * 16 + i] = E::pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1]));
-        if (p.o_f32 && row < p.N) {   // the values whose rounding O is
+        if (kVariants && p.o_f32 && row < p.N) {   // the values whose rounding O is
           uint4* dst = reinterpret_cast<uint4*>(p.o_f32 + (size_t(w.bh) * p.N + row) * D + c * 32);
 #pragma unroll
           for (int i = 0; i < 8; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
@@ -542,9 +554,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(ow[4 * i], ow[4 * i + 1], ow[4 * i + 2], ow[4 * i + 3]);
         p.lse[size_t(w.bh) * p.N + row] = (ms + (raised ? p.delta_log2 : 0.f) + lg2(l)) * kLn2;
-        if (p.ties)
+        if (kVariants && p.ties)
           p.ties[size_t(w.bh) * p.N + row] = cnt | (raised ? (1 << 29) : 0) | (ever_repeated ? (1 << 30) : 0);
-        if (p.one_hit) p.one_hit[size_t(w.bh) * p.N + row] = hits;
+        if (kVariants && p.one_hit) p.one_hit[size_t(w.bh) * p.N + row] = hits;
       }
       it_cnt += n_t;
     }
