@@ -166,11 +166,16 @@ BIAS_INPUTS = [("gpt2m", {}), ("long", {"B": 32, "H": 12, "N": 2048})]
 
 
 def test_bias_on_repeated_maxima(fa):
-    """Pass for fix_mode 1: |z| < 3 for the mean and the magnitude-aligned
-    mean error over repeated-max rows, and |aligned mean| <= 2^-12 mean|O|.
-    Power: fix_mode 3 puts the maxima off the bf16 grid (P_bar 0.9375 where
-    l holds 0.9394) and must be seen shrinking |O|.  fix_mode 0 is measured
-    and printed beside them."""
+    """Pass for fix_mode 1: the mean error and the magnitude-aligned mean error
+    over repeated-max rows are bounded, |mean| + 3 SE <= 2^-14 mean|O| (1/32 of
+    bf16's half step 2^-9): the sign-coherent error the fix targets stays far
+    below what a bf16 output could show, with 3-sigma confidence at any sample
+    size.  Power: fix_mode 3 puts the maxima off the bf16 grid (P_bar 0.9375
+    where l holds 0.9394) and must be seen outside the same bound, shrinking
+    |O|.  fix_mode 0 is measured and printed beside them, with the paired
+    difference of the two modes on the same rows.  (A bare |z| < 3 would not
+    do: over a few hundred thousand rows every mode, the self-normalised one
+    included, shows a common FP32 shrink of about 1e-6 mean|O|.)"""
     from flashattention_bf16_fwd_b200.stats import bias_stats
     from oracle import attention_fwd
 
@@ -206,13 +211,22 @@ def test_bias_on_repeated_maxima(fa):
             stats[(m, kind)] = bias_stats(np.concatenate(sel[m][kind]), ref, rows)
         cr = np.concatenate(ctrl_ref)
         stats[(m, "control_f32")] = bias_stats(np.concatenate(ctrl[m]), cr, np.ones(cr.shape[0], bool))
+    a0 = np.mean(np.sign(ref) * (np.concatenate(sel[0]["f32"]) - ref), axis=-1)
+    a1 = np.mean(np.sign(ref) * (np.concatenate(sel[1]["f32"]) - ref), axis=-1)
+    dpair = a0 - a1
+    print(f"bias paired aligned fix_mode 0 - 1: {dpair.mean() / np.abs(ref).mean():+.2e} mean|O|, "
+          f"z {dpair.mean() / (dpair.std(ddof=1) / np.sqrt(dpair.size)):+.2f}")
     for key, s in stats.items():
         print(f"bias fix_mode {key[0]} {key[1]}: rows {s['rows']} z_mean {s['z_mean']:+.2f} "
               f"z_aligned {s['z_aligned']:+.2f} aligned/mean|O| {s['aligned_mean'] / s['mean_abs_ref']:+.2e}")
-    s1 = stats[(1, "f32")]
-    assert abs(s1["z_mean"]) < 3 and abs(s1["z_aligned"]) < 3, s1
-    assert abs(s1["aligned_mean"]) <= 2.0 ** -12 * s1["mean_abs_ref"], s1
+    bound = 2.0 ** -14
+
+    def within(st):
+        m = st["mean_abs_ref"]
+        return (abs(st["mean"]) + 3 * st["se_mean"] <= bound * m and
+                abs(st["aligned_mean"]) + 3 * st["se_aligned"] <= bound * m)
+
+    assert within(stats[(1, "f32")]), stats[(1, "f32")]
+    assert within(stats[(1, "control_f32")]), stats[(1, "control_f32")]
     s3 = stats[(3, "f32")]
-    assert s3["z_aligned"] < -5, s3
-    c1 = stats[(1, "control_f32")]
-    assert abs(c1["z_mean"]) < 3 and abs(c1["z_aligned"]) < 3, c1
+    assert s3["aligned_mean"] + 3 * s3["se_aligned"] < -bound * s3["mean_abs_ref"], s3
