@@ -175,20 +175,6 @@ constexpr CUtensorMapDataType map_type() {
 // H query heads share Hkv key/value heads (H == Hkv: ordinary attention).
 int check_heads(int H, int Hkv) { return (Hkv >= 1 && Hkv <= H && H % Hkv == 0) ? FA_OK : FA_ERR_SHAPE; }
 
-// The kernels schedule their work items in groups of heads whose streamed
-// tensors fit in half of the 126 MB L2 together.
-constexpr double kL2GroupBytes = 64.0 * (1 << 20);
-
-// Heads per scheduling group when each head streams `bytes_per_head`: all of
-// them when they fit together, else the fewest equal groups that fit.
-int heads_per_group(double bytes_per_head, int heads) {
-  const double total = bytes_per_head * heads;
-  if (total <= kL2GroupBytes) return heads;
-  const long long groups = (long long)std::ceil(total / kL2GroupBytes);
-  const long long hg = (heads + groups - 1) / groups;
-  return hg < 1 ? 1 : int(hg);
-}
-
 template <typename E>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int32_t* ties, int32_t* one_hit,
                float* o_f32, int B, int H, int Hkv, int N, int d, int causal, float scale, int fix_mode,
@@ -219,8 +205,6 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   prm.BH = BH;
   prm.N = N;
   prm.n_pairs = (N + 255) / 256;
-  // a query head streams K and V (shared by the H / Hkv heads of its group)
-  prm.hg = heads_per_group(4.0 * N * d / (H / Hkv), BH);
   prm.causal = causal;
   prm.scale_log2 = float(double(scale) * 1.4426950408889634);
   // shift on repeated-max rows per fix_mode, in base-2 units: 1 and 5 map the
@@ -326,9 +310,6 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse,
   prm.dv = dv;
   prm.dev_error = st->dev_error;
   prm.BH = BHkv;   // work items run over the K/V heads
-  // a K/V head streams Q and dO (2 bytes each) and the FP32 dQ accumulator of
-  // each of its H / Hkv query heads
-  prm.hg = heads_per_group(8.0 * N * d * (H / Hkv), BHkv);
   prm.H = H;
   prm.group = H / Hkv;
   prm.N = N;

@@ -87,7 +87,6 @@ struct BwdParams {
   int* dev_error;
   int BH, N, n_kv, causal;   // BH = batch * K/V heads
   int H, group;         // query heads per batch entry; query heads per K/V head (1 = no sharing)
-  int hg;               // K/V heads per scheduling group (their Q, dO and dQ fit in the L2 together)
   float scale, scale_log2;
 };
 
@@ -141,22 +140,17 @@ struct BwdLayout {
 // One work item = one (batch*K/V head, 128-key tile).  It loops over the
 // query tiles that see those keys, for each query head of the group that
 // shares the K/V head (dK, dV accumulate over all of them): n_it steps.
-// Items are numbered in groups of hg K/V heads whose Q, dO and dQ accumulator
-// fit in the L2 together; within a group heavy first (causal: the first key
-// tiles are seen by the most query tiles).  CTAs are persistent and sweep the
-// items with snake_item().
+// Items are numbered heavy first (causal: the first key tiles are seen by the
+// most query tiles); CTAs are persistent and sweep the sorted items with
+// snake_item().
 struct BwdItem {
   int bh, kv_tile, key0, i_start, n_it_head, n_it;
 };
 
 __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
   BwdItem w;
-  const int per_group = p.hg * p.n_kv;
-  const int grp = item / per_group;
-  const int j = item - grp * per_group;
-  const int hg = min(p.hg, p.BH - grp * p.hg);   // the last group may be smaller
-  w.kv_tile = j / hg;
-  w.bh = grp * p.hg + (j - w.kv_tile * hg);
+  w.kv_tile = item / p.BH;
+  w.bh = item % p.BH;
   w.key0 = w.kv_tile * 128;
   const int n_q = (p.N + 127) / 128;
   w.i_start = p.causal ? w.kv_tile : 0;
@@ -394,24 +388,38 @@ __global__ void __launch_bounds__(512, 1)
         auto wait_do = [&](uint32_t gg) {
           return mbar_wait(&do_full[gg % L::kDOStages], (gg / L::kDOStages) & 1, wd);
         };
+        // K and V of the item started n items ago (start-address halves)
+        auto k_of = [&](uint32_t n) {
+          return (smem_u32(smem + L::kKVOff) >> 4) + (n % L::kKVStages) * (2 * L::kTileBytes >> 4);
+        };
         uint32_t g = 0;        // query-tile steps issued
         uint32_t n_done = 0;   // items started
         bool ok = true;
+        // d = 64 holds two items' K and V: the next item's first S^T and dP^T
+        // are issued during this item's last step (as within an item), so
+        // the compute warps do not wait for them at the item boundary
+        bool first_issued = false;
         for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
           const BwdItem w = bwd_item(p, item);
           const uint32_t ks = n_done % L::kKVStages;
-          const uint32_t sk = (smem_u32(smem + L::kKVOff) >> 4) + ks * (2 * L::kTileBytes >> 4);
+          const uint32_t sk = k_of(n_done);
           const uint32_t sv = sk + (L::kTileBytes >> 4);
-          if (!(ok = mbar_wait(&kv_full[ks], (n_done / L::kKVStages) & 1, wd) && wait_q(g) && wait_do(g))) break;
-          tc_fence_after();
-          kmajor_mma(tmem + L::kTmS, sk, q_of(g));     // S^T = K Q^T of the item's first query tile
-          umma_commit(s_full);
-          if (L::kWide && g > 0) {                      // the previous dQ shares the dP^T columns
-            if (!(ok = mbar_wait(dq_free, (g - 1) & 1, wd))) break;
+          const bool prefetch_next = !L::kWide && snake_item(rnd + 1) < n_items;
+          const uint32_t nsk = k_of(n_done + 1);
+          const uint32_t nsv = nsk + (L::kTileBytes >> 4);
+          if (!first_issued) {
+            if (!(ok = mbar_wait(&kv_full[ks], (n_done / L::kKVStages) & 1, wd) && wait_q(g) && wait_do(g))) break;
             tc_fence_after();
+            kmajor_mma(tmem + L::kTmS, sk, q_of(g));     // S^T = K Q^T of the item's first query tile
+            umma_commit(s_full);
+            if (L::kWide && g > 0) {                      // the previous dQ shares the dP^T columns
+              if (!(ok = mbar_wait(dq_free, (g - 1) & 1, wd))) break;
+              tc_fence_after();
+            }
+            kmajor_mma(tmem + L::kTmDP, sv, do_of(g));   // dP^T = V dO^T
+            umma_commit(dp_full);
           }
-          kmajor_mma(tmem + L::kTmDP, sv, do_of(g));   // dP^T = V dO^T
-          umma_commit(dp_full);
+          first_issued = false;
           // the first dV/dK MMA of an item overwrites the accumulators: the
           // previous item's epilogue must have read them
           if (!(ok = mbar_wait(dkv_free, (n_done & 1) ^ 1, wd))) break;
@@ -430,6 +438,13 @@ __global__ void __launch_bounds__(512, 1)
               if (!(ok = wait_q(g + 1))) break;
               tc_fence_after();
               kmajor_mma(tmem + L::kTmS, sk, q_of(g + 1));
+              umma_commit(s_full);
+            } else if (prefetch_next) {                 // the next item's first S^T, with its K
+              if (!(ok = mbar_wait(&kv_full[(n_done + 1) % L::kKVStages], ((n_done + 1) / L::kKVStages) & 1, wd) &&
+                         wait_q(g + 1)))
+                break;
+              tc_fence_after();
+              kmajor_mma(tmem + L::kTmS, nsk, q_of(g + 1));
               umma_commit(s_full);
             }
             if (!(ok = mbar_wait(ds_full, g & 1, wd))) break;
@@ -457,6 +472,12 @@ __global__ void __launch_bounds__(512, 1)
               tc_fence_after();
               kmajor_mma(tmem + L::kTmDP, sv, do_of(g + 1));
               umma_commit(dp_full);
+            } else if (prefetch_next) {                 // the next item's first dP^T, with its V
+              if (!(ok = wait_do(g + 1))) break;
+              tc_fence_after();
+              kmajor_mma(tmem + L::kTmDP, nsv, do_of(g + 1));
+              umma_commit(dp_full);
+              first_issued = true;
             }
           }
           umma_commit(&kv_empty[ks]);                   // K and V of this item are no longer read

@@ -20,7 +20,7 @@
 //   warps 10-11 idle (they complete the third warpgroup)
 // Registers: launched at 168 per thread (384 threads); the third warpgroup
 // gives back down to 88 and the two softmax warpgroups take 208 each:
-// 128 * (208 + 208 + 88) = 384 * 168.
+// 128 * (208 + 208 + 88) = 384 * 168 (d = 128: 200, 200 and 104).
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 after.
 // P_bar (bf16 or fp16, two per 32-bit column) overwrites the first 64 columns of S_t
 // and is the A operand of O_t += P_bar V (V is the MN-major B operand).
@@ -41,7 +41,6 @@ struct FwdParams {
   int* dev_error;       // library error flag
   int BH, N, n_pairs, causal;   // BH = batch * query heads
   int H, group;         // query heads per batch entry; query heads per K/V head (1 = no sharing)
-  int hg;               // heads per scheduling group (their K/V fit in the L2 together)
   float scale_log2;     // scale * log2(e): S -> base-2 exponent domain
   float delta_log2;     // shift added to m on repeated-max rows (0 = fix off)
   float fix_factor;     // 2^-delta_log2: P at a repeated maximum (1 - 2^-8 or, in fp16, 1 - 2^-11; 0.5; exp(-1/16))
@@ -72,29 +71,26 @@ struct FwdLayout {
   __host__ __device__ static constexpr uint32_t tm_o(int t) { return kSepP ? 384 + 64 * t : 256 + D * t; }
   static constexpr int kThreads = 384;
   static constexpr int kLaunchRegs = 168;       // per thread, fixed by __launch_bounds__(384, 1)
-  static constexpr uint32_t kSoftmaxRegs = 208;
-  static constexpr uint32_t kOtherRegs = 88;
+  // d = 128 moves 8 registers per thread from the softmax warpgroups to the
+  // producer/MMA warpgroup, whose longer MMA sequences spilled at 88
+  static constexpr uint32_t kSoftmaxRegs = (D == 128) ? 200 : 208;
+  static constexpr uint32_t kOtherRegs = (D == 128) ? 104 : 88;
   static_assert(128 * (2 * kSoftmaxRegs + kOtherRegs) <= kThreads * kLaunchRegs, "register split exceeds the pool");
 };
 
 // One work item = one (batch*head, pair of query tiles).  Items are numbered
-// in groups of hg heads whose K/V fit in the L2 together, so that the CTAs in
-// flight stream few heads at once; within a group heavy first (causal: the
-// last query tiles see the most keys).  The CTAs are persistent and sweep the
-// items with snake_item().
+// heavy first (causal: the last query tiles see the most keys); the CTAs are
+// persistent and sweep the sorted items with snake_item().  (Grouping the
+// items by heads so that fewer heads' K/V stream through the L2 at once was
+// measured slower: the balance of the heavy-first order matters more.)
 struct FwdItem {
   int bh, q0_row, n0, n1, nmax;
 };
 
 __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
   FwdItem it;
-  const int per_group = p.hg * p.n_pairs;
-  const int grp = item / per_group;
-  const int j = item - grp * per_group;
-  const int hg = min(p.hg, p.BH - grp * p.hg);   // the last group may be smaller
-  const int rank = j / hg;
-  it.bh = grp * p.hg + (j - rank * hg);
-  const int pair = p.causal ? (p.n_pairs - 1 - rank) : rank;
+  const int pair = p.causal ? (p.n_pairs - 1 - item / p.BH) : item / p.BH;
+  it.bh = item % p.BH;
   it.q0_row = pair * 256;
   const int n_kv = (p.N + 127) / 128;
   it.n0 = p.causal ? min(2 * pair + 1, n_kv) : n_kv;
@@ -409,10 +405,19 @@ __global__ void __launch_bounds__(384, 1)
         // equal to the tile max ride along as independent packed adds
         uint64_t sum2[4] = {0, 0, 0, 0};
         uint64_t eq2[2] = {0, 0};
+        const uint64_t sl2_2 = f2_pack(sl2, sl2);
+        const uint64_t nmsh_2 = f2_pack(-msh, -msh);
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          const float x0 = fmaf(s[2 * i], sl2, -msh);
-          const float x1 = fmaf(s[2 * i + 1], sl2, -msh);
+          // x = S * scale_log2 - shift: one packed FMA per pair at d = 128; at
+          // d = 64 the packed form pushes the softmax past its register budget
+          float x0, x1;
+          if constexpr (D == 128) {
+            f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), sl2_2, nmsh_2), x0, x1);
+          } else {
+            x0 = fmaf(s[2 * i], sl2, -msh);
+            x1 = fmaf(s[2 * i + 1], sl2, -msh);
+          }
           const float e0 = (s[2 * i] == mt) ? 1.f : 0.f;
           const float e1 = (s[2 * i + 1] == mt) ? 1.f : 0.f;
           eq2[i & 1] = f2_add(eq2[i & 1], f2_pack(e0, e1));
