@@ -186,7 +186,8 @@ struct BwdSteps {
 //   warp  12    producer: K, V per item; Q_i (TMA) plus LSE_i, D_i per step,
 //               up to kQStages steps ahead
 //   warp  14    producer: dO_i (TMA), independent of the Q ring
-//   warp  13    TMEM allocator + tcgen05.mma issuer
+//   warp  13    TMEM allocator + tcgen05.mma issuer (the whole warp runs the
+//               issuing loop; one elected lane executes each instruction)
 //   warp  15    idle (completes the fourth warpgroup)
 // MMA order per query tile i (the tensor core runs the next tile's S while
 // the CUDA cores form dS_i, and dK_i, dQ_i, dP_{i+1} while they form P_{i+1}):
@@ -355,12 +356,14 @@ __global__ void __launch_bounds__(512, 1)
       }
     } else if (warp == 13) {
       // ---------------------------------------------------------- MMA issuer
-      if (lane == 0) {
+      // The whole warp runs this loop (warp-uniform operands and waits); one
+      // elected lane executes each tcgen05.mma and tcgen05.commit.
+      {
         constexpr uint32_t kIdS = make_idesc(128, 128, 0, 0, E::kMmaFmt);   // K Q^T, V dO^T: K-major operands
         constexpr uint32_t kIdAcc = make_idesc(128, D, 0, 1, E::kMmaFmt);   // TMEM A x MN-major B (dV, dK)
         constexpr uint32_t kIdDQ = make_idesc(128, D, 1, 1, E::kMmaFmt);    // dS (MN-major) x K (MN-major)
         // Descriptors as 32-bit low halves with one shared high half (every
-        // operand has a 1024-byte stride): this thread shares its issue slots
+        // operand has a 1024-byte stride): this warp shares its issue slots
         // with the busiest warps of the CTA, so each MMA costs it only an add.
         // K-major operands use a leading byte offset of 16, MN-major ones the
         // distance between 64-wide blocks.
@@ -372,7 +375,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t off = ((k >> 2) * L::kSubBytes + (k & 3) * 32) >> 4;
-            umma_ss_lh(d_tm, (a_lo + off) | kLboK, (b_lo + off) | kLboK, kHi, kIdS, k > 0 ? 1u : 0u);
+            umma_ss_lh_warp(d_tm, (a_lo + off) | kLboK, (b_lo + off) | kLboK, kHi, kIdS, k > 0 ? 1u : 0u);
           }
         };
         // start-address halves (address >> 4) of each buffer
@@ -383,10 +386,10 @@ __global__ void __launch_bounds__(512, 1)
           return (smem_u32(smem + L::kDOOff) >> 4) + (gg % L::kDOStages) * (L::kTileBytes >> 4);
         };
         auto wait_q = [&](uint32_t gg) {
-          return mbar_wait(&q_full[gg % L::kQStages], (gg / L::kQStages) & 1, wd);
+          return __all_sync(0xffffffffu, mbar_wait(&q_full[gg % L::kQStages], (gg / L::kQStages) & 1, wd));
         };
         auto wait_do = [&](uint32_t gg) {
-          return mbar_wait(&do_full[gg % L::kDOStages], (gg / L::kDOStages) & 1, wd);
+          return __all_sync(0xffffffffu, mbar_wait(&do_full[gg % L::kDOStages], (gg / L::kDOStages) & 1, wd));
         };
         // K and V of the item started n items ago (start-address halves)
         auto k_of = [&](uint32_t n) {
@@ -408,83 +411,83 @@ __global__ void __launch_bounds__(512, 1)
           const uint32_t nsk = k_of(n_done + 1);
           const uint32_t nsv = nsk + (L::kTileBytes >> 4);
           if (!first_issued) {
-            if (!(ok = mbar_wait(&kv_full[ks], (n_done / L::kKVStages) & 1, wd) && wait_q(g) && wait_do(g))) break;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[ks], (n_done / L::kKVStages) & 1, wd)) && wait_q(g) && wait_do(g))) break;
             tc_fence_after();
             kmajor_mma(tmem + L::kTmS, sk, q_of(g));     // S^T = K Q^T of the item's first query tile
-            umma_commit(s_full);
+            umma_commit_warp(s_full);
             if (L::kWide && g > 0) {                      // the previous dQ shares the dP^T columns
-              if (!(ok = mbar_wait(dq_free, (g - 1) & 1, wd))) break;
+              if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_free, (g - 1) & 1, wd)))) break;
               tc_fence_after();
             }
             kmajor_mma(tmem + L::kTmDP, sv, do_of(g));   // dP^T = V dO^T
-            umma_commit(dp_full);
+            umma_commit_warp(dp_full);
           }
           first_issued = false;
           // the first dV/dK MMA of an item overwrites the accumulators: the
           // previous item's epilogue must have read them
-          if (!(ok = mbar_wait(dkv_free, (n_done & 1) ^ 1, wd))) break;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(dkv_free, (n_done & 1) ^ 1, wd)))) break;
           for (int it = 0; ok && it < w.n_it; ++it, ++g) {
             const uint32_t sq = q_of(g);
             const uint32_t sdo = do_of(g);
-            if (!(ok = mbar_wait(p_full, g & 1, wd))) break;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_full, g & 1, wd)))) break;
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < 8; ++k)                 // dV += P_bar^T dO_i
-              umma_ts_lh(tmem + L::kTmDV, tmem + L::pt_col(k), (sdo + k * (2048 >> 4)) | kLboMN, kHi, kIdAcc,
+              umma_ts_lh_warp(tmem + L::kTmDV, tmem + L::pt_col(k), (sdo + k * (2048 >> 4)) | kLboMN, kHi, kIdAcc,
                          (it > 0 || k > 0) ? 1u : 0u);
-            umma_commit(pt_free);
-            umma_commit(&do_empty[g % L::kDOStages]);   // dP_i and dV_i were the readers of dO_i
+            umma_commit_warp(pt_free);
+            umma_commit_warp(&do_empty[g % L::kDOStages]);   // dP_i and dV_i were the readers of dO_i
             if (it + 1 < w.n_it) {                      // S^T_{i+1}
               if (!(ok = wait_q(g + 1))) break;
               tc_fence_after();
               kmajor_mma(tmem + L::kTmS, sk, q_of(g + 1));
-              umma_commit(s_full);
+              umma_commit_warp(s_full);
             } else if (prefetch_next) {                 // the next item's first S^T, with its K
-              if (!(ok = mbar_wait(&kv_full[(n_done + 1) % L::kKVStages], ((n_done + 1) / L::kKVStages) & 1, wd) &&
+              if (!(ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[(n_done + 1) % L::kKVStages], ((n_done + 1) / L::kKVStages) & 1, wd)) &&
                          wait_q(g + 1)))
                 break;
               tc_fence_after();
               kmajor_mma(tmem + L::kTmS, nsk, q_of(g + 1));
-              umma_commit(s_full);
+              umma_commit_warp(s_full);
             }
-            if (!(ok = mbar_wait(ds_full, g & 1, wd))) break;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_full, g & 1, wd)))) break;
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < 8; ++k)                 // dK += dS^T Q_i
-              umma_ts_lh(tmem + L::kTmDK, tmem + L::dst_col(k), (sq + k * (2048 >> 4)) | kLboMN, kHi, kIdAcc,
+              umma_ts_lh_warp(tmem + L::kTmDK, tmem + L::dst_col(k), (sq + k * (2048 >> 4)) | kLboMN, kHi, kIdAcc,
                          (it > 0 || k > 0) ? 1u : 0u);
             if (!L::kWide && g > 0) {                   // the drain has read dQ of the previous step
-              if (!(ok = mbar_wait(dq_free, (g - 1) & 1, wd))) break;
+              if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_free, (g - 1) & 1, wd)))) break;
               tc_fence_after();
             }
 #pragma unroll
             for (int k = 0; k < 8; ++k)                 // dQ_i = dS K
-              umma_ss_lh(tmem + L::kTmDQ, ds_lo + k * (2048 >> 4), (sk + k * (2048 >> 4)) | kLboMN, kHi, kIdDQ,
+              umma_ss_lh_warp(tmem + L::kTmDQ, ds_lo + k * (2048 >> 4), (sk + k * (2048 >> 4)) | kLboMN, kHi, kIdDQ,
                          k > 0 ? 1u : 0u);
-            umma_commit(dq_full);
-            umma_commit(&q_empty[g % L::kQStages]);
+            umma_commit_warp(dq_full);
+            umma_commit_warp(&q_empty[g % L::kQStages]);
             if (it + 1 < w.n_it) {                      // dP^T_{i+1}
               if (L::kWide) {                           // dQ_i shares the dP^T columns
-                if (!(ok = mbar_wait(dq_free, g & 1, wd))) break;
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_free, g & 1, wd)))) break;
                 tc_fence_after();
               }
               if (!(ok = wait_do(g + 1))) break;
               tc_fence_after();
               kmajor_mma(tmem + L::kTmDP, sv, do_of(g + 1));
-              umma_commit(dp_full);
+              umma_commit_warp(dp_full);
             } else if (prefetch_next) {                 // the next item's first dP^T, with its V
               if (!(ok = wait_do(g + 1))) break;
               tc_fence_after();
               kmajor_mma(tmem + L::kTmDP, nsv, do_of(g + 1));
-              umma_commit(dp_full);
+              umma_commit_warp(dp_full);
               first_issued = true;
             }
           }
-          umma_commit(&kv_empty[ks]);                   // K and V of this item are no longer read
-          umma_commit(dkv_done);                        // dK, dV of this item are final
+          umma_commit_warp(&kv_empty[ks]);                   // K and V of this item are no longer read
+          umma_commit_warp(dkv_done);                        // dK, dV of this item are final
         }
-        umma_commit(mma_done);
-        mbar_wait(mma_done, 0, wd);
+        umma_commit_warp(mma_done);
+        __all_sync(0xffffffffu, mbar_wait(mma_done, 0, wd));
       }
       __syncwarp();
     }
@@ -640,28 +643,35 @@ __global__ void __launch_bounds__(512, 1)
         // TMEM -> swizzled 32 x 32 FP32 box in shared memory -> TMA reduce-add
         // into the FP32 accumulator (rows past N are dropped by the TMA unit)
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_dq + c * 32, r);
-          tmem_ld_wait(r);
-          if (c == D / 32 - 1) {                       // dQ is in registers: its TMEM may be reused
+        for (int c2 = 0; c2 < D / 64; ++c2) {          // two 32-column chunks per TMEM wait: dQ's
+                                                       // columns are released sooner (d = 128: dP waits on them)
+          uint32_t r[2][32];
+          tmem_ld32(t_dq + (2 * c2) * 32, r[0]);
+          tmem_ld32(t_dq + (2 * c2 + 1) * 32, r[1]);
+          tmem_ld_wait(r[0]);
+          tmem_ld_wait(r[1]);
+          if (c2 == D / 64 - 1) {                      // dQ is in registers: its TMEM may be reused
             tc_fence_before();
             mbar_arrive(dq_free);
           }
-          uint8_t* box = stage + (box_seq & 1) * L::kStageBox;
-          if (lane == 0) bulk_wait_read<1>();          // the reduce issued from this box is done reading
-          __syncwarp();
 #pragma unroll
-          for (int c16 = 0; c16 < 8; ++c16)
-            *reinterpret_cast<uint4*>(box + lane * 128 + ((c16 ^ (lane & 7)) << 4)) =
-                make_uint4(r[4 * c16], r[4 * c16 + 1], r[4 * c16 + 2], r[4 * c16 + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_reduce_add_3d(&tm_dq, box, c * 32, sp.qt * 128 + wq * 32, sp.bh_q);
-            bulk_commit();
+          for (int h = 0; h < 2; ++h) {
+            const int c = 2 * c2 + h;
+            uint8_t* box = stage + (box_seq & 1) * L::kStageBox;
+            if (lane == 0) bulk_wait_read<1>();        // the reduce issued from this box is done reading
+            __syncwarp();
+#pragma unroll
+            for (int c16 = 0; c16 < 8; ++c16)
+              *reinterpret_cast<uint4*>(box + lane * 128 + ((c16 ^ (lane & 7)) << 4)) =
+                  make_uint4(r[h][4 * c16], r[h][4 * c16 + 1], r[h][4 * c16 + 2], r[h][4 * c16 + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_reduce_add_3d(&tm_dq, box, c * 32, sp.qt * 128 + wq * 32, sp.bh_q);
+              bulk_commit();
+            }
+            ++box_seq;
           }
-          ++box_seq;
         }
       }
       if (!ok) break;

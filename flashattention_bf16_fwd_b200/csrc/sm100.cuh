@@ -280,6 +280,45 @@ __device__ __forceinline__ void umma_ts_lh(uint32_t d_tmem, uint32_t a_tmem, uin
       : "memory");
 }
 
+// The same three instructions issued by a whole warp: every lane runs the
+// issuing loop with the same operand values, which then stay warp-uniform,
+// and one lane, elected in the instruction's own block, executes it.  Issued
+// from a single lane inside a divergent branch instead, each MMA cost the
+// backward's issuer 70-100 cycles.
+__device__ __forceinline__ void umma_ss_lh_warp(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred P, E;\n\t.reg .b64 A, B;\n\t"
+      "elect.sync _|E, 0xffffffff;\n\t"
+      "setp.ne.b32 P, %5, 0;\n\t"
+      "mov.b64 A, {%1, %3};\n\t"
+      "mov.b64 B, {%2, %3};\n\t"
+      "@E tcgen05.mma.cta_group::1.kind::f16 [%0], A, B, %4, P;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_ts_lh_warp(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred P, E;\n\t.reg .b64 B;\n\t"
+      "elect.sync _|E, 0xffffffff;\n\t"
+      "setp.ne.b32 P, %5, 0;\n\t"
+      "mov.b64 B, {%2, %3};\n\t"
+      "@E tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], B, %4, P;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred E;\n\t"
+      "elect.sync _|E, 0xffffffff;\n\t"
+      "@E tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
 // A descriptor advanced by `bytes` along its start address (bits 0-13 hold
 // address >> 4; shared-memory addresses stay below 256 KB, so no carry
 // leaves the field).
