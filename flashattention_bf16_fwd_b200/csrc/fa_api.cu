@@ -80,10 +80,14 @@ DeviceState* device_state(int* why = nullptr) {
     setup(fa_fwd_kernel<128, false, ElemF16>, FwdLayout<128>::kAlloc, FwdLayout<128>::kLaunchRegs);
     setup(fa_fwd_kernel<64, true, ElemF16>, FwdLayout<64>::kAlloc, FwdLayout<64>::kLaunchRegs);
     setup(fa_fwd_kernel<128, true, ElemF16>, FwdLayout<128>::kAlloc, FwdLayout<128>::kLaunchRegs);
-    setup(fa_bwd_kernel<64, ElemBF16>, BwdLayout<64>::kAlloc, BwdLayout<64>::kLaunchRegs);
-    setup(fa_bwd_kernel<128, ElemBF16>, BwdLayout<128>::kAlloc, BwdLayout<128>::kLaunchRegs);
-    setup(fa_bwd_kernel<64, ElemF16>, BwdLayout<64>::kAlloc, BwdLayout<64>::kLaunchRegs);
-    setup(fa_bwd_kernel<128, ElemF16>, BwdLayout<128>::kAlloc, BwdLayout<128>::kLaunchRegs);
+    setup(fa_bwd_kernel<64, ElemBF16, false>, BwdLayout<64>::kAlloc, BwdLayout<64>::kLaunchRegs);
+    setup(fa_bwd_kernel<128, ElemBF16, false>, BwdLayout<128>::kAlloc, BwdLayout<128>::kLaunchRegs);
+    setup(fa_bwd_kernel<64, ElemF16, false>, BwdLayout<64>::kAlloc, BwdLayout<64>::kLaunchRegs);
+    setup(fa_bwd_kernel<128, ElemF16, false>, BwdLayout<128>::kAlloc, BwdLayout<128>::kLaunchRegs);
+    setup(fa_bwd_kernel<64, ElemBF16, true>, BwdLayout<64>::kAlloc, BwdLayout<64>::kLaunchRegs);
+    setup(fa_bwd_kernel<128, ElemBF16, true>, BwdLayout<128>::kAlloc, BwdLayout<128>::kLaunchRegs);
+    setup(fa_bwd_kernel<64, ElemF16, true>, BwdLayout<64>::kAlloc, BwdLayout<64>::kLaunchRegs);
+    setup(fa_bwd_kernel<128, ElemF16, true>, BwdLayout<128>::kAlloc, BwdLayout<128>::kLaunchRegs);
     st->status = !ok ? FA_ERR_DEVICE : !regs_ok ? FA_ERR_BUILD : FA_OK;
   });
   if (st->status != FA_OK) {
@@ -310,6 +314,13 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse,
   prm.dv = dv;
   prm.dev_error = st->dev_error;
   prm.BH = BHkv;   // work items run over the K/V heads
+  // Head-major pairs of key tiles when the heads the default (key-tile major)
+  // order keeps in flight would stream more than half the L2 together: each
+  // K/V head streams Q and dO (2 bytes an element) and the FP32 dQ
+  // accumulator of each of its H / Hkv query heads.
+  const double per_head = 8.0 * N * d * (H / Hkv);
+  const double in_flight = BHkv < st->num_sms ? BHkv : st->num_sms;
+  const bool pairs = in_flight * per_head > 64.0 * (1 << 20);
   prm.H = H;
   prm.group = H / Hkv;
   prm.N = N;
@@ -320,11 +331,10 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse,
   const int n_items = prm.n_kv * BHkv;
   const dim3 grid(unsigned(n_items < st->num_sms ? n_items : st->num_sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const cudaError_t e =
-      (d == 64) ? launch(fa_bwd_kernel<64, E>, grid, dim3(BwdLayout<64>::kThreads), BwdLayout<64>::kAlloc, s, mq, mk,
-                         mv, mdo, mdq, prm)
-                : launch(fa_bwd_kernel<128, E>, grid, dim3(BwdLayout<128>::kThreads), BwdLayout<128>::kAlloc, s, mq,
-                         mk, mv, mdo, mdq, prm);
+  auto kern = (d == 64) ? (pairs ? fa_bwd_kernel<64, E, true> : fa_bwd_kernel<64, E, false>)
+                        : (pairs ? fa_bwd_kernel<128, E, true> : fa_bwd_kernel<128, E, false>);
+  const int smem = (d == 64) ? BwdLayout<64>::kAlloc : BwdLayout<128>::kAlloc;
+  const cudaError_t e = launch(kern, grid, dim3(BwdLayout<64>::kThreads), smem, s, mq, mk, mv, mdo, mdq, prm);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 

@@ -140,24 +140,62 @@ struct BwdLayout {
 // One work item = one (batch*K/V head, 128-key tile).  It loops over the
 // query tiles that see those keys, for each query head of the group that
 // shares the K/V head (dK, dV accumulate over all of them): n_it steps.
-// Items are numbered heavy first (causal: the first key tiles are seen by the
-// most query tiles); CTAs are persistent and sweep the sorted items with
-// snake_item().
 struct BwdItem {
   int bh, kv_tile, key0, i_start, n_it_head, n_it;
 };
 
-__device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
+__device__ __forceinline__ BwdItem bwd_item_at(const BwdParams& p, int bh, int kv_tile) {
   BwdItem w;
-  w.kv_tile = item / p.BH;
-  w.bh = item % p.BH;
-  w.key0 = w.kv_tile * 128;
+  w.bh = bh;
+  w.kv_tile = kv_tile;
+  w.key0 = kv_tile * 128;
   const int n_q = (p.N + 127) / 128;
-  w.i_start = p.causal ? w.kv_tile : 0;
+  w.i_start = p.causal ? kv_tile : 0;
   w.n_it_head = n_q - w.i_start;
   w.n_it = w.n_it_head * p.group;
   return w;
 }
+
+// The sequence of work items a persistent CTA takes; every role of the CTA
+// walks the same sequence.
+//  - Default: items are numbered heavy first, key tile major (causal: the
+//    first key tiles are seen by the most query tiles), and the CTAs sweep
+//    them with snake_item().  All CTAs work on different heads at once.
+//  - pairs: a unit is one head and two key tiles t and n_kv - 1 - t, taken
+//    one after the other by the same CTA.  Under a causal mask every pair
+//    has the same number of steps (n_q + 1), so the units can be numbered
+//    head major without unbalancing the CTAs, and the CTAs in flight cover
+//    only about 148 / (n_kv / 2) heads: their Q, dO and FP32 dQ accumulator
+//    then stay in the L2 instead of being streamed again for every key tile.
+//    The host chooses it (a separate kernel instantiation) when the heads the
+//    default order keeps in flight would not fit in the L2 together.
+template <bool kPairs>
+struct BwdSched {
+  int rnd, sub, item, per_head, n_units;
+  __device__ __forceinline__ explicit BwdSched(const BwdParams& p) : rnd(0), sub(0), item(snake_item(0)) {
+    per_head = kPairs ? (p.n_kv + 1) / 2 : p.n_kv;
+    n_units = per_head * p.BH;
+  }
+  __device__ __forceinline__ bool valid() const { return item < n_units; }
+  __device__ __forceinline__ BwdItem get(const BwdParams& p) const {
+    if constexpr (!kPairs) {
+      return bwd_item_at(p, item % p.BH, item / p.BH);
+    } else {
+      const int pp = item % per_head;
+      return bwd_item_at(p, item / per_head, sub ? p.n_kv - 1 - pp : pp);
+    }
+  }
+  __device__ __forceinline__ void next(const BwdParams& p) {
+    if constexpr (kPairs) {
+      if (sub == 0 && 2 * (item % per_head) + 1 != p.n_kv) {   // a lone middle tile has no second
+        sub = 1;
+        return;
+      }
+      sub = 0;
+    }
+    item = snake_item(++rnd);
+  }
+};
 
 // The steps of an item in order: query tile qt of batch*query-head bh_q,
 // query tiles innermost.  Advanced once per step, without divisions.
@@ -195,8 +233,8 @@ struct BwdSteps {
 // Barrier phases run on per-CTA counters, so items follow one another without
 // re-initialisation: `g` counts query-tile steps, `n_done` counts items.
 // E: the element format (ElemBF16 or ElemF16) of Q, K, V, dO, dK, dV and of
-// the P_bar and dS operands.
-template <int D, typename E = ElemBF16>
+// the P_bar and dS operands.  kPairs: the head-major pair schedule (BwdSched).
+template <int D, typename E = ElemBF16, bool kPairs = false>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -230,7 +268,6 @@ __global__ void __launch_bounds__(512, 1)
     if (threadIdx.x == 0) atomicExch(p.dev_error, kDevErrSmemAlign);
     return;
   }
-  const int n_items = p.n_kv * p.BH;
   const int warp = int(warp_id());
   const int lane = int(lane_id());
 
@@ -290,8 +327,8 @@ __global__ void __launch_bounds__(512, 1)
       uint32_t g = 0;        // query-tile steps loaded
       uint32_t n_done = 0;   // items started
       bool ok = true;
-      for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
-        const BwdItem w = bwd_item(p, item);
+      for (BwdSched<kPairs> sc(p); ok && sc.valid(); sc.next(p), ++n_done) {
+        const BwdItem w = sc.get(p);
         const uint32_t ks = n_done % L::kKVStages;
         ok = __all_sync(0xffffffffu, mbar_wait(&kv_empty[ks], ((n_done / L::kKVStages) & 1) ^ 1, wd));
         if (!ok) break;
@@ -336,8 +373,8 @@ __global__ void __launch_bounds__(512, 1)
       const uint64_t pol_q = l2_policy_evict_last();
       uint32_t g = 0;
       bool ok = true;
-      for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd)) {
-        const BwdItem w = bwd_item(p, item);
+      for (BwdSched<kPairs> sc(p); ok && sc.valid(); sc.next(p)) {
+        const BwdItem w = sc.get(p);
         BwdSteps sp(p, w);
         for (int it = 0; it < w.n_it; ++it, ++g, sp.next()) {
           const int q0 = sp.qt * 128;
@@ -402,12 +439,14 @@ __global__ void __launch_bounds__(512, 1)
         // are issued during this item's last step (as within an item), so
         // the compute warps do not wait for them at the item boundary
         bool first_issued = false;
-        for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
-          const BwdItem w = bwd_item(p, item);
+        for (BwdSched<kPairs> sc(p); ok && sc.valid(); sc.next(p), ++n_done) {
+          const BwdItem w = sc.get(p);
           const uint32_t ks = n_done % L::kKVStages;
           const uint32_t sk = k_of(n_done);
           const uint32_t sv = sk + (L::kTileBytes >> 4);
-          const bool prefetch_next = !L::kWide && snake_item(rnd + 1) < n_items;
+          BwdSched<kPairs> nx = sc;
+          nx.next(p);
+          const bool prefetch_next = !L::kWide && nx.valid();
           const uint32_t nsk = k_of(n_done + 1);
           const uint32_t nsv = nsk + (L::kTileBytes >> 4);
           if (!first_issued) {
@@ -505,8 +544,8 @@ __global__ void __launch_bounds__(512, 1)
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     uint32_t g = 0;
     bool ok = true;
-    for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd)) {
-      const BwdItem w = bwd_item(p, item);
+    for (BwdSched<kPairs> sc(p); ok && sc.valid(); sc.next(p)) {
+      const BwdItem w = sc.get(p);
       const bool key_in = w.key0 + kr < p.N;
       BwdSteps sp(p, w);
       for (int it = 0; it < w.n_it; ++it, ++g, sp.next()) {
@@ -633,8 +672,8 @@ __global__ void __launch_bounds__(512, 1)
     uint32_t g = 0;
     uint32_t n_done = 0;
     bool ok = true;
-    for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
-      const BwdItem w = bwd_item(p, item);
+    for (BwdSched<kPairs> sc(p); ok && sc.valid(); sc.next(p), ++n_done) {
+      const BwdItem w = sc.get(p);
       BwdSteps sp(p, w);
       for (int it = 0; it < w.n_it; ++it, ++g, sp.next()) {
         ok = __all_sync(0xffffffffu, mbar_wait(dq_full, g & 1, wd));
