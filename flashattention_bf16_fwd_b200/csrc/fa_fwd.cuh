@@ -353,7 +353,8 @@ __global__ void __launch_bounds__(384, 1)
       float l = 0.f;        // running sum of the unrounded P, relative to the shift in use
       bool ever_repeated = false;   // the running max occurred >= 2 times at some tile
       float l_bar = 0.f;    // running sum of the rounded P_bar (self-normalised mode only)
-      int cnt_near = 0;     // entries whose P rounds to 1 under the current shift (near-tie mode)
+      int cnt_near = 0;     // near-tie mode: 2 when two or more entries so far have P rounding to 1 under the plain shift
+      float s2 = kNegInf;   // near-tie mode: second largest raw score so far (a repeated maximum counts twice)
       int hits = 0;         // entries packed as P_bar == 1.0 since the shift last moved (one_hit record)
 
       for (int j = 0; j < n_t; ++j) {
@@ -392,6 +393,12 @@ __global__ void __launch_bounds__(384, 1)
         const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
         const float m_new = fmaxf(m, mt);
         const float ms_new = (m_new == kNegInf) ? 0.f : m_new * sl2;
+        // near-tie mode: the largest score of the tile below its maximum
+        float s2x = kNegInf;
+        if (kVariants && p.near) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) s2x = fmaxf(s2x, (s[i] < mt) ? s[i] : kNegInf);
+        }
 
         // A row whose running maximum is already repeated and does not move in
         // this tile keeps the raised shift whatever the tile holds, so its P
@@ -430,15 +437,17 @@ __global__ void __launch_bounds__(384, 1)
         const int ct = (mt == kNegInf) ? 0 : int(ea + eb);
         int c_new = (m == m_new ? cnt : 0) + (mt == m_new ? ct : 0);
         if (m_new == kNegInf) c_new = 0;
-        // near-tie mode: entries of this tile whose P (plain shift) rounds to
-        // 1.0 in the element format (P >= 1 - 2^-9 in bf16, 1 - 2^-12 in
-        // fp16); earlier tiles' count stands while the shift has not moved
+        // near-tie mode: the row has two or more entries whose P under the
+        // plain shift rounds to 1.0 in the element format (P >= 1 - 2^-9 in
+        // bf16, 1 - 2^-12 in fp16) exactly when its second largest score
+        // does; the two largest scores are carried across key tiles, so
+        // partners in earlier tiles still count after the maximum moves
         int cn_new = 0;
+        float s2_new = kNegInf;
         if (kVariants && p.near) {
-          int cn = 0;
-#pragma unroll
-          for (int i = 0; i < 128; ++i) cn += (s[i] >= rounds_to_one<E>()) ? 1 : 0;
-          cn_new = (m == m_new ? cnt_near : 0) + cn;
+          const float s2t = (ct >= 2) ? mt : s2x;
+          s2_new = (m > mt) ? fmaxf(s2, mt) : ((mt > m) ? fmaxf(m, s2t) : mt);
+          cn_new = (s2_new != kNegInf && ex2(fmaf(s2_new, sl2, -ms_new)) >= rounds_to_one<E>()) ? 2 : 0;
         }
         const int det = (kVariants && p.near) ? cn_new : c_new;
         ever_repeated |= (det >= 2);
@@ -525,6 +534,7 @@ __global__ void __launch_bounds__(384, 1)
         m = m_new;
         cnt = c_new;
         cnt_near = cn_new;
+        s2 = s2_new;
         ms = ms_new;
         raised = raise;
       }

@@ -91,9 +91,8 @@ typedef enum {
  *                     sum of the rounded P_bar (self-normalised);
  *                 5 = fix_mode 1 triggered by near ties: two or more entries
  *                     whose P (plain shift) rounds to bf16 1.0, i.e.
- *                     P >= 1 - 2^-9.  Counted per key tile under the shift in
- *                     use; a count from earlier tiles is dropped when the row
- *                     maximum moves.
+ *                     P >= 1 - 2^-9, over the whole row (the two largest
+ *                     scores are carried across key tiles).
  *                 LSE is the unrounded log-sum-exp in every mode.
  * Returns FA_OK or a negative fa_status.
  */
