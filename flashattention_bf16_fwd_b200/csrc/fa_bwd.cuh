@@ -254,7 +254,6 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* dq_free = bars + 13;
   uint64_t* dkv_done = bars + 14;
   uint64_t* dkv_free = bars + 15;
-  uint64_t* pt_free = bars + 16;
   uint64_t* mma_done = bars + 17;
   uint64_t* q_full = bars + 18;    // [kQStages]
   uint64_t* q_empty = bars + 21;   // [kQStages]
@@ -290,7 +289,6 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(dq_free, 128);
     mbar_init(dkv_done, 1);
     mbar_init(dkv_free, 128);
-    mbar_init(pt_free, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -474,7 +472,6 @@ __global__ void __launch_bounds__(512, 1)
             for (int k = 0; k < 8; ++k)                 // dV += P_bar^T dO_i
               umma_ts_lh_warp(tmem + L::kTmDV, tmem + L::pt_col(k), (sdo + k * (2048 >> 4)) | kLboMN, kHi, kIdAcc,
                          (it > 0 || k > 0) ? 1u : 0u);
-            umma_commit_warp(pt_free);
             umma_commit_warp(&do_empty[g % L::kDOStages]);   // dP_i and dV_i were the readers of dO_i
             if (it + 1 < w.n_it) {                      // S^T_{i+1}
               if (!(ok = wait_q(g + 1))) break;
@@ -593,10 +590,9 @@ __global__ void __launch_bounds__(512, 1)
             }
           }
         }
-        if (!L::kWide && g > 0) {                      // dV of the previous step has read P_bar^T
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(pt_free, (g - 1) & 1, wd)))) break;
-          tc_fence_after();
-        }
+        // No wait before overwriting P_bar^T: dV of the previous step, its
+        // last reader, was issued before this step's S^T, and the tensor core
+        // completes one thread's MMAs in order, so s_full implies it is done.
         {
           uint32_t wv[16];
 #pragma unroll
@@ -645,10 +641,9 @@ __global__ void __launch_bounds__(512, 1)
           for (int i = 0; i < 16; ++i) wv[i] = dsw[16 + i];
           tmem_st16(t_dp + 16, wv);
         }
-        // dS into shared memory for dQ = dS K: MN-major, 128-byte swizzle
-        if (g > 0) {                                   // dQ of the previous step has read it
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_full, (g - 1) & 1, wd)))) break;
-        }
+        // dS into shared memory for dQ = dS K: MN-major, 128-byte swizzle.
+        // dQ of the previous step, its last reader, was issued before this
+        // step's dP^T, so dp_full already implied that it is done.
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) {
           uint4* dst = reinterpret_cast<uint4*>(ds_row + ((c16 ^ (kr & 7)) << 4));
