@@ -80,3 +80,42 @@ def test_gqa_with_one_group_per_head_is_plain_attention(fa):
     torch.cuda.synchronize()
     assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
     assert normwise_rel_err(dq1.float().cpu().numpy(), dq2.float().cpu().numpy().astype(np.float64)) < 2.0 ** -8
+
+
+def test_gqa_at_a_size_that_takes_the_pair_schedule(fa):
+    """B=6, H=32 query heads over Hkv=8 key/value heads, N=1024, d=64, causal.
+    The backward's heads in flight (48 key/value heads, each with its group's
+    Q, dO and FP32 dQ rows: 2 MiB) exceed the 64 MiB the host allows for the
+    L2, so the backward runs the head-major pair schedule (key tiles t and
+    n_kv-1-t of one head, each over the four query heads of its group).  Two
+    sampled key/value heads, with their query heads, against the oracle."""
+    B, H, Hkv, N, d = 6, 32, 8, 1024, 64
+    g = H // Hkv
+    q, k, v, do = draw(B, H, Hkv, N, d, seed=77)
+    scale = d ** -0.5
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o = torch.empty_like(qd)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    assert fa.fa_fwd_ex(qd, kd, vd, o, lse, True, scale, 1) == 0
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    assert fa.fa_bwd_ex(qd, kd, vd, o, lse, dod, dq, dk, dv, ws, True, scale) == 0
+    torch.cuda.synchronize()
+    assert fa.fa_check_device_error() == 0
+    for b, hk in ((0, 0), (5, 7)):
+        hq = slice(hk * g, (hk + 1) * g)
+        qs, dos = q[b:b + 1, hq], do[b:b + 1, hq]
+        ks, vs = k[b:b + 1, hk:hk + 1], v[b:b + 1, hk:hk + 1]
+        ke, ve = gqa_expand(ks, g), gqa_expand(vs, g)
+        o_ref, lse_ref = attention_fwd(qs, ke, ve, True, scale)
+        assert np.abs(o[b:b + 1, hq].float().cpu().numpy() - o_ref).max() <= O_ATOL
+        assert lse_rel_err(lse[b:b + 1, hq].cpu().numpy(), lse_ref) <= LSE_RTOL
+        dq_ref, dk_rep, dv_rep = attention_bwd(qs, ke, ve, dos, True, scale)
+        refs = {"dq": (dq[b:b + 1, hq], dq_ref), "dk": (dk[b:b + 1, hk:hk + 1], gqa_reduce(dk_rep, g)),
+                "dv": (dv[b:b + 1, hk:hk + 1], gqa_reduce(dv_rep, g))}
+        for name, (got, ref) in refs.items():
+            err = normwise_rel_err(got.float().cpu().numpy(), ref)
+            assert err <= GRAD_RTOL, (b, hk, name, err)
+    for t in (o, lse, dq, dk, dv):
+        assert torch.isfinite(t).all()
