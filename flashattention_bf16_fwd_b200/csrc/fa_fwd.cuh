@@ -10,17 +10,27 @@
 // exponent, the maxima included, is strictly below 1.
 //
 // Persistent CTAs (one per SM) loop over work items; one item = one
-// (batch, head) and two 128-row query tiles, processed in ping-pong so the
-// tensor core works on one tile while the other tile's softmax runs on the
-// CUDA cores.  An item's epilogue overlaps the next item's first MMAs:
-//   warps 0-3  softmax of query tile 0 (thread r owns row r: TMEM lane r)
-//   warps 4-7  softmax of query tile 1
-//   warp  8    TMA producer: Q tiles once, then a ring of K/V stages
-//   warp  9    TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 10-11 idle (they complete the third warpgroup)
+// (batch, head) and two 128-row query tiles, processed by two softmax
+// warpgroups so the tensor core works on one tile while the other tile's
+// softmax runs on the CUDA cores.  An item's epilogue overlaps the next item's
+// first MMAs:
+//   warps 0-3  softmax warpgroup 0 (thread r owns row r: TMEM lane r)
+//   warps 4-7  softmax warpgroup 1
+//   warp  8    TMA producer: an item's Q tiles, then a ring of K/V stages
+//   warp  9    TMEM allocator + tcgen05.mma issuer (single thread); at d = 64
+//              it issues warpgroup 0's MMAs only
+//   warp 10    d = 64: tcgen05.mma issuer of warpgroup 1 (idle at d = 128)
+//   warp 11    idle (it completes the third warpgroup)
+// d = 64 runs the two warpgroups' MMA chains independently, each with its own
+// issuer and its own walk over the items, and keeps two Q buffers: under a
+// causal mask the second query tile of an item sees one key tile more than the
+// first, so the warpgroup that takes it alternates from one item to the next
+// (odd rounds swap the tiles), and the warpgroup with the shorter tile starts
+// the next item instead of waiting.  d = 128 has room for neither and keeps
+// one issuer that alternates the warpgroups tile by tile.
 // Registers: launched at 168 per thread (384 threads); the third warpgroup
-// gives back down to 88 and the two softmax warpgroups take 208 each:
-// 128 * (208 + 208 + 88) = 384 * 168 (d = 128: 200, 200 and 104).
+// gives back down to 104 and the two softmax warpgroups take 200 each:
+// 128 * (200 + 200 + 104) = 384 * 168.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 after.
 // P_bar (bf16 or fp16, two per 32-bit column) overwrites the first 64 columns of S_t
 // and is the A operand of O_t += P_bar V (V is the MN-major B operand).
@@ -55,8 +65,9 @@ struct FwdLayout {
   static constexpr int kSub = D / 64;                 // 64-column sub-tiles per 128-row tile
   static constexpr int kSubBytes = 128 * 64 * 2;      // one TMA box, 16 KB
   static constexpr int kTileBytes = kSub * kSubBytes; // a 128 x D bf16 tile
-  static constexpr int kQOff = 0;                     // Q0, Q1
-  static constexpr int kKVOff = 2 * kTileBytes;       // stage s: K, then V
+  static constexpr int kQBufs = (D == 64) ? 2 : 1;    // Q buffers (d = 64: the next item's Q loads early)
+  static constexpr int kQOff = 0;                     // buffer b: the tiles of warpgroups 0 and 1
+  static constexpr int kKVOff = kQBufs * 2 * kTileBytes;   // stage s: K, then V
   static constexpr int kBarOff = kKVOff + kStages * 2 * kTileBytes;
   static constexpr int kBytes = kBarOff + 256;
   static constexpr int kAlloc = kBytes + 1024;        // room to align the base to 1 KB
@@ -71,10 +82,10 @@ struct FwdLayout {
   __host__ __device__ static constexpr uint32_t tm_o(int t) { return kSepP ? 384 + 64 * t : 256 + D * t; }
   static constexpr int kThreads = 384;
   static constexpr int kLaunchRegs = 168;       // per thread, fixed by __launch_bounds__(384, 1)
-  // d = 128 moves 8 registers per thread from the softmax warpgroups to the
-  // producer/MMA warpgroup, whose longer MMA sequences spilled at 88
-  static constexpr uint32_t kSoftmaxRegs = (D == 128) ? 200 : 208;
-  static constexpr uint32_t kOtherRegs = (D == 128) ? 104 : 88;
+  // the producer/MMA warpgroup spills below 104 (d = 128: longer MMA
+  // sequences; d = 64: two issuers)
+  static constexpr uint32_t kSoftmaxRegs = 200;
+  static constexpr uint32_t kOtherRegs = 104;
   static_assert(128 * (2 * kSoftmaxRegs + kOtherRegs) <= kThreads * kLaunchRegs, "register split exceeds the pool");
 };
 
@@ -97,6 +108,14 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
   it.n1 = (it.q0_row + 128 < p.N) ? (p.causal ? min(2 * pair + 2, n_kv) : n_kv) : 0;
   it.nmax = max(it.n0, it.n1);
   return it;
+}
+
+// The query tile (0 or 1 of the item) that softmax warpgroup t takes in round
+// rnd of the CTA's item walk.  d = 64 swaps them in odd rounds, so that the
+// longer causal tile alternates between the warpgroups.
+template <int D>
+__device__ __forceinline__ int fwd_tile_of(int t, int rnd) {
+  return FwdLayout<D>::kSepP ? (t ^ (rnd & 1)) : t;
 }
 
 // The smallest value below 1 that rounds to 1.0 in E's format (ties to even):
@@ -122,17 +141,17 @@ __global__ void __launch_bounds__(384, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* q_full = bars;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;
+  uint64_t* q_full = bars;         // [kQBufs]
+  uint64_t* q_empty = bars + 2;    // [kQBufs]
+  uint64_t* kv_full = bars + 4;
   uint64_t* kv_empty = kv_full + L::kStages;
   uint64_t* s_full = kv_empty + L::kStages;  // [2]
   uint64_t* p_full = s_full + 2;             // [2]
   uint64_t* o_done = p_full + 2;             // [2]
   uint64_t* o_free = o_done + 2;             // [2]
   uint64_t* s_free = o_free + 2;             // [2] the softmax has read S_t (d = 64)
-  uint64_t* mma_done = s_free + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* mma_done = s_free + 2;          // [2] one per MMA issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int n_items = p.n_pairs * p.BH;
@@ -140,11 +159,13 @@ __global__ void __launch_bounds__(384, 1)
   const int lane = int(lane_id());
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    for (int b = 0; b < L::kQBufs; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_empty[b], L::kSepP ? 2 : 1);   // d = 64: both MMA issuers
+    }
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], L::kSepP ? 2 : 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
@@ -153,7 +174,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&o_free[t], 128);
       mbar_init(&s_free[t], 128);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(&mma_done[0], 1);
+    mbar_init(&mma_done[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -191,14 +213,15 @@ __global__ void __launch_bounds__(384, 1)
           const FwdItem w = fwd_item(p, item);
           // grouped-query layout: query head h reads K/V head h / group
           const int kv_bh = (w.bh / p.H) * (p.H / p.group) + (w.bh % p.H) / p.group;
-          // the previous item's S MMAs must be done with Q
-          if (!(ok = mbar_wait(q_empty, (n_done & 1) ^ 1, wd))) break;
+          // the S MMAs of the item kQBufs back must be done with this Q buffer
+          const uint32_t qb = n_done % L::kQBufs;
+          if (!(ok = mbar_wait(&q_empty[qb], ((n_done / L::kQBufs) & 1) ^ 1, wd))) break;
           const int nq = (w.n1 > 0) ? 2 : 1;
-          mbar_arrive_expect_tx(q_full, uint32_t(nq * L::kTileBytes));
-          for (int t = 0; t < nq; ++t)
+          mbar_arrive_expect_tx(&q_full[qb], uint32_t(nq * L::kTileBytes));
+          for (int qt = 0; qt < nq; ++qt)   // query tile qt into the buffer of the warpgroup that takes it
             for (int s = 0; s < L::kSub; ++s)
-              tma_load_3d(smem + L::kQOff + t * L::kTileBytes + s * L::kSubBytes, &tm_q, q_full, s * 64,
-                          w.q0_row + t * 128, w.bh, pol_q);
+              tma_load_3d(smem + L::kQOff + (qb * 2 + fwd_tile_of<D>(qt, rnd)) * L::kTileBytes + s * L::kSubBytes,
+                          &tm_q, &q_full[qb], s * 64, w.q0_row + qt * 128, w.bh, pol_q);
           for (int j = 0; j < w.nmax; ++j, ++kv_cnt) {
             const uint32_t st = kv_cnt % L::kStages;
             if (!(ok = mbar_wait(&kv_empty[st], ((kv_cnt / L::kStages) & 1) ^ 1, wd))) break;
@@ -212,8 +235,89 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
+    } else if (L::kSepP && (warp == 9 || warp == 10)) {
+      // ------------------------------------------ d = 64: MMA issuers, one per
+      // softmax warpgroup, each walking the items on its own.  Q buffers and
+      // K/V stages are released once both issuers are done with them (their
+      // empty barriers count two arrivals); a warpgroup whose tile of an item
+      // is shorter goes on to the next item while the other finishes.
+      if (lane == 0) {
+        const int t = warp - 9;
+        constexpr uint32_t kIdS = make_idesc(128, 128, 0, 0, E::kMmaFmt);
+        constexpr uint32_t kIdPV = make_idesc(128, D, 0, 1, E::kMmaFmt);
+        const uint64_t dq0 = make_sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
+        const uint64_t dk0 = make_sdesc_sw128(smem_u32(smem + L::kKVOff), 16, 1024);
+        const uint64_t dv0 = make_sdesc_sw128(smem_u32(smem + L::kKVOff + L::kTileBytes), L::kSubBytes, 1024);
+        uint32_t qb = 0;
+        auto issue_s = [&](uint32_t st) {
+          const uint64_t a = sdesc_add(dq0, (qb * 2 + t) * L::kTileBytes);
+          const uint64_t b = sdesc_add(dk0, st * 2 * L::kTileBytes);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k >> 2) * L::kSubBytes + (k & 3) * 32;
+            umma_ss(tmem + L::tm_s(t), sdesc_add(a, off), sdesc_add(b, off), kIdS, k > 0);
+          }
+          umma_commit(&s_full[t]);
+        };
+        auto issue_pv = [&](uint32_t st, int j) {
+          const uint64_t b = sdesc_add(dv0, st * 2 * L::kTileBytes);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_ts(tmem + L::tm_o(t), tmem + L::tm_p(t) + k * 8, sdesc_add(b, k * 2048), kIdPV,
+                    (j > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&o_done[t]);
+        };
+        uint32_t kv_cnt = 0, it_cnt = 0, ep_cnt = 0, n_done = 0;
+        bool ok = true;
+        for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
+          const FwdItem w = fwd_item(p, item);
+          const int nt = fwd_tile_of<D>(t, rnd) ? w.n1 : w.n0;   // key tiles of this warpgroup's query tile
+          qb = n_done % L::kQBufs;
+          if (!(ok = mbar_wait(&q_full[qb], (n_done / L::kQBufs) & 1, wd))) break;
+          if (nt > 0) {
+            if (!(ok = mbar_wait(&kv_full[kv_cnt % L::kStages], (kv_cnt / L::kStages) & 1, wd))) break;
+            if (it_cnt > 0 && !(ok = mbar_wait(&s_free[t], (it_cnt - 1) & 1, wd))) break;
+            tc_fence_after();
+            issue_s(kv_cnt % L::kStages);
+          }
+          if (nt <= 1) umma_commit(&q_empty[qb]);   // this issuer's S MMAs of the item are issued
+          for (int j = 0; ok && j < w.nmax; ++j) {
+            const uint32_t st = (kv_cnt + j) % L::kStages;
+            if (j + 1 < nt) {
+              const uint32_t nxt = kv_cnt + j + 1;
+              if (!(ok = mbar_wait(&kv_full[nxt % L::kStages], (nxt / L::kStages) & 1, wd) &&
+                         mbar_wait(&s_free[t], (it_cnt + j) & 1, wd)))
+                break;
+              tc_fence_after();
+              issue_s(nxt % L::kStages);
+              if (j + 2 == nt) umma_commit(&q_empty[qb]);
+            }
+            if (j < nt) {
+              if (!(ok = mbar_wait(&p_full[t], (it_cnt + j) & 1, wd))) break;
+              if (j == 0 && !(ok = mbar_wait(&o_free[t], (ep_cnt & 1) ^ 1, wd))) break;
+              tc_fence_after();
+              issue_pv(st, j);
+            }
+            // a key tile this warpgroup does not use (its query tile sees
+            // fewer): wait until it is loaded before releasing its stage, so
+            // that this issuer's arrival belongs to this use of the stage and
+            // it never runs a use ahead of the other issuer
+            if (j >= nt && !(ok = mbar_wait(&kv_full[st], ((kv_cnt + j) / L::kStages) & 1, wd))) break;
+            umma_commit(&kv_empty[st]);          // this issuer is done with the stage
+          }
+          kv_cnt += w.nmax;
+          it_cnt += nt;
+          ep_cnt += (nt > 0) ? 1 : 0;
+        }
+        umma_commit(&mma_done[t]);
+        mbar_wait(&mma_done[t], 0, wd);
+      }
+      __syncwarp();
     } else if (warp == 9) {
-      // ---------------------------------------------------------- MMA issuer
+      // ---------------------------------------- d = 128: MMA issuer (one thread)
+      // Per key tile j: P_bar_0 V, S_0 of tile j+1 (it overwrites P_bar_0),
+      // P_bar_1 V, S_1 of tile j+1; the two warpgroups alternate at the
+      // tensor core.
       if (lane == 0) {
         constexpr uint32_t kIdS = make_idesc(128, 128, 0, 0, E::kMmaFmt);   // Q K^T: both K-major
         constexpr uint32_t kIdPV = make_idesc(128, D, 0, 1, E::kMmaFmt);    // P_bar V: V is MN-major
@@ -251,33 +355,14 @@ __global__ void __launch_bounds__(384, 1)
                      mbar_wait(&kv_full[kv_cnt % L::kStages], (kv_cnt / L::kStages) & 1, wd)))
             break;
           tc_fence_after();
-          for (int t = 0; t < 2; ++t) {
-            if (nt[t] == 0) continue;
-            // d=64: the softmax must have read the last S_t of the previous item
-            if (L::kSepP && it_cnt[t] > 0 && !(ok = mbar_wait(&s_free[t], (it_cnt[t] - 1) & 1, wd))) break;
-            issue_s(t, kv_cnt % L::kStages);
-          }
-          if (ok && w.nmax == 1) umma_commit(q_empty);
+          for (int t = 0; t < 2; ++t)
+            if (nt[t] > 0) issue_s(t, kv_cnt % L::kStages);
+          if (w.nmax == 1) umma_commit(q_empty);
           for (int j = 0; ok && j < w.nmax; ++j) {
             const uint32_t st = (kv_cnt + j) % L::kStages;
             const uint32_t stn = (kv_cnt + j + 1) % L::kStages;
-            if (L::kSepP) {
-              // S of key tile j+1 as soon as the softmax has read S of tile j;
-              // then P_bar V of tile j
-              if (j + 1 < w.nmax) {
-                const uint32_t nxt = kv_cnt + j + 1;
-                if (!(ok = mbar_wait(&kv_full[stn], (nxt / L::kStages) & 1, wd))) break;
-                for (int t = 0; t < 2; ++t) {
-                  if (j + 1 >= nt[t]) continue;
-                  if (!(ok = mbar_wait(&s_free[t], (it_cnt[t] + j) & 1, wd))) break;
-                  tc_fence_after();
-                  issue_s(t, stn);
-                }
-                if (!ok) break;
-                if (j + 2 == w.nmax) umma_commit(q_empty);   // the item's last S MMAs are issued
-              }
-              for (int t = 0; t < 2; ++t) {
-                if (j >= nt[t]) continue;
+            for (int t = 0; t < 2; ++t) {
+              if (j < nt[t]) {
                 if (!(ok = mbar_wait(&p_full[t], (it_cnt[t] + j) & 1, wd))) break;
                 // the first P_bar V of an item overwrites O_t: the previous
                 // item's epilogue must have read it
@@ -285,27 +370,16 @@ __global__ void __launch_bounds__(384, 1)
                 tc_fence_after();
                 issue_pv(t, st, j);
               }
-              if (!ok) break;
-              umma_commit(&kv_empty[st]);
-            } else {
-              for (int t = 0; t < 2; ++t) {
-                if (j < nt[t]) {
-                  if (!(ok = mbar_wait(&p_full[t], (it_cnt[t] + j) & 1, wd))) break;
-                  if (j == 0 && !(ok = mbar_wait(&o_free[t], (ep_cnt[t] & 1) ^ 1, wd))) break;
-                  tc_fence_after();
-                  issue_pv(t, st, j);
-                }
-                if (t == 0 && j + 1 < w.nmax) {
-                  const uint32_t nxt = kv_cnt + j + 1;
-                  if (!(ok = mbar_wait(&kv_full[stn], (nxt / L::kStages) & 1, wd))) break;
-                  tc_fence_after();
-                  if (j + 1 < nt[0]) issue_s(0, stn);   // S_0 of tile j+1 overwrites P_bar_0 after P_bar V
-                }
-                if (t == 1) {
-                  umma_commit(&kv_empty[st]);
-                  if (j + 1 < nt[1]) issue_s(1, stn);
-                  if (j + 2 == w.nmax) umma_commit(q_empty);   // the item's last S MMAs are issued
-                }
+              if (t == 0 && j + 1 < w.nmax) {
+                const uint32_t nxt = kv_cnt + j + 1;
+                if (!(ok = mbar_wait(&kv_full[stn], (nxt / L::kStages) & 1, wd))) break;
+                tc_fence_after();
+                if (j + 1 < nt[0]) issue_s(0, stn);   // S_0 of tile j+1 overwrites P_bar_0 after P_bar V
+              }
+              if (t == 1) {
+                umma_commit(&kv_empty[st]);
+                if (j + 1 < nt[1]) issue_s(1, stn);
+                if (j + 2 == w.nmax) umma_commit(q_empty);   // the item's last S MMAs are issued
               }
             }
           }
@@ -316,8 +390,8 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         // Every MMA must be finished before TMEM is released.
-        umma_commit(mma_done);
-        mbar_wait(mma_done, 0, wd);
+        umma_commit(&mma_done[0]);
+        mbar_wait(&mma_done[0], 0, wd);
       }
       __syncwarp();
     }
@@ -341,9 +415,10 @@ __global__ void __launch_bounds__(384, 1)
 
     for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd)) {
       const FwdItem w = fwd_item(p, item);
-      const int n_t = t ? w.n1 : w.n0;
+      const int qt = fwd_tile_of<D>(t, rnd);   // which of the item's two query tiles
+      const int n_t = qt ? w.n1 : w.n0;
       if (n_t == 0) continue;
-      const int row = w.q0_row + t * 128 + (warp & 3) * 32 + lane;
+      const int row = w.q0_row + qt * 128 + (warp & 3) * 32 + lane;
       const int limit = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
 
       float m = kNegInf;    // running max of the raw scores S
