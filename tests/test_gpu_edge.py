@@ -118,3 +118,38 @@ def test_tiny_scale(fa):
     assert abs(float(g["lse"][0, 0, 499]) - math.log(500)) < 1e-2
     for name, ref in zip(("dq", "dk", "dv"), attention_bwd(x["q"], x["k"], x["v"], x["do"], True, 1e-3)):
         assert normwise_rel_err(g[name], ref) <= GRAD_RTOL, name
+
+
+REPEAT_CASES = [(2, 3, 777, 64, True), (1, 4, 1000, 64, True), (3, 2, 129, 64, True), (2, 2, 700, 128, True),
+                (1, 3, 333, 64, False)]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", REPEAT_CASES,
+                         ids=[f"B{b}H{h}N{n}d{d}{'c' if c else 'f'}" for b, h, n, d, c in REPEAT_CASES])
+def test_forward_repeats_bit_for_bit(fa, B, H, N, d, causal):
+    """The forward is deterministic: 40 back-to-back calls give the same O,
+    LSE and tie record, bit for bit, and no bounded wait expires.  At d = 64
+    the two softmax warpgroups run independent MMA chains that share the K/V
+    stages and the Q buffers; a release that raced ahead of the other chain
+    would let a stage be refilled while still in use, and show here as a
+    changed output or an expired wait.  The shapes include items with a
+    single query tile and odd tails."""
+    x = make_inputs(Workload("rep", B, H, N, d, causal=causal), seed=N + d + B)
+    dev = torch.device("cuda")
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    o0, l0, t0 = fa.attention_fwd(q, k, v, causal=causal, scale=x["scale"], fix_mode=1, ties=True)
+    outs = []
+    for _ in range(40):
+        outs.append(fa.attention_fwd(q, k, v, causal=causal, scale=x["scale"], fix_mode=1, ties=True))
+    torch.cuda.synchronize()
+    assert fa.fa_check_device_error() == 0
+    for o, l, t in outs:
+        assert torch.equal(o, o0) and torch.equal(l, l0) and torch.equal(t, t0)
+    # the production instantiation (no records) as well
+    p0 = fa.attention_fwd(q, k, v, causal=causal, scale=x["scale"], fix_mode=1)
+    for _ in range(40):
+        o, l = fa.attention_fwd(q, k, v, causal=causal, scale=x["scale"], fix_mode=1)
+        assert torch.equal(o, p0[0]) and torch.equal(l, p0[1])
+    torch.cuda.synchronize()
+    assert fa.fa_check_device_error() == 0
+    assert torch.equal(p0[0], o0) and torch.equal(p0[1], l0)
