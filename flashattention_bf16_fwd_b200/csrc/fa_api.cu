@@ -137,15 +137,17 @@ int check_common(int B, int H, int N, int d, int causal, float scale) {
   return FA_OK;
 }
 
-// A [BH, N, D] bf16 tensor seen as 3-D (d, n, bh); boxes of 64 x 128 x 1 with
-// the 128-byte swizzle the tcgen05 descriptors expect.  Rows past N read 0.
+// A [BH, N, D] bf16 tensor seen as 3-D (d, n, bh); boxes of 64 x box_rows x 1
+// (128 for the loads the tcgen05 descriptors read, 32 for the forward's O
+// stores, one per warp) with the 128-byte swizzle.  Loads read 0 past N; stores
+// drop rows past N.
 bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D,
-              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, unsigned box_rows = 128) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(N), cuuint64_t(BH)};
   cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(N) * D * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -192,10 +194,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if (fix_mode < 0 || fix_mode > 5) return FA_ERR_FIXMODE;
   FA_DEVICE_OR_RETURN(st);
   const int BH = B * H;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   constexpr CUtensorMapDataType dt = map_type<E>();
   if (!make_map(&mq, q, BH, N, d, dt) || !make_map(&mk, k, B * Hkv, N, d, dt) ||
-      !make_map(&mv, v, B * Hkv, N, d, dt))
+      !make_map(&mv, v, B * Hkv, N, d, dt) || !make_map(&mo, o, BH, N, d, dt, 32))
     return FA_ERR_DEVICE;
   FwdParams prm{};
   prm.H = H;
@@ -230,7 +232,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   auto kern = (d == 64) ? (variants ? fa_fwd_kernel<64, true, E> : fa_fwd_kernel<64, false, E>)
                         : (variants ? fa_fwd_kernel<128, true, E> : fa_fwd_kernel<128, false, E>);
   const int smem = (d == 64) ? FwdLayout<64>::kAlloc : FwdLayout<128>::kAlloc;
-  const cudaError_t e = launch(kern, grid, dim3(FwdLayout<64>::kThreads), smem, stream, mq, mk, mv, prm);
+  const cudaError_t e = launch(kern, grid, dim3(FwdLayout<64>::kThreads), smem, stream, mq, mk, mv, mo, prm);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 

@@ -21,6 +21,9 @@
 //              it issues warpgroup 0's MMAs only
 //   warp 10    d = 64: tcgen05.mma issuer of warpgroup 1 (idle at d = 128)
 //   warp 11    idle (it completes the third warpgroup)
+// d = 64 stores O through a 128-byte-swizzled staging tile per warpgroup: each
+// warp writes its 32 rows there and issues one TMA store box, so the softmax
+// warps move on to the next item instead of issuing row-wise global stores.
 // d = 64 runs the two warpgroups' MMA chains independently, each with its own
 // issuer and its own walk over the items, and keeps two Q buffers: under a
 // causal mask the second query tile of an item sees one key tile more than the
@@ -68,7 +71,11 @@ struct FwdLayout {
   static constexpr int kQBufs = (D == 64) ? 2 : 1;    // Q buffers (d = 64: the next item's Q loads early)
   static constexpr int kQOff = 0;                     // buffer b: the tiles of warpgroups 0 and 1
   static constexpr int kKVOff = kQBufs * 2 * kTileBytes;   // stage s: K, then V
-  static constexpr int kBarOff = kKVOff + kStages * 2 * kTileBytes;
+  // d = 64: O leaves through a swizzled staging tile per warpgroup (TMA store
+  // of one 32-row box per warp)
+  static constexpr int kOOff = kKVOff + kStages * 2 * kTileBytes;
+  static constexpr int kOStage = (D == 64) ? 2 * kTileBytes : 0;
+  static constexpr int kBarOff = kOOff + kOStage;
   static constexpr int kBytes = kBarOff + 256;
   static constexpr int kAlloc = kBytes + 1024;        // room to align the base to 1 KB
   static constexpr uint32_t kTmemCols = 512;
@@ -133,7 +140,8 @@ __device__ __forceinline__ constexpr float rounds_to_one() {
 template <int D, bool kVariants, typename E = ElemBF16>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const FwdParams p) {
   using L = FwdLayout<D>;
   const float kNegInf = -__int_as_float(0x7f800000);
   constexpr float kLn2 = 0.69314718055994531f;
@@ -639,10 +647,28 @@ __global__ void __launch_bounds__(384, 1)
       // O_t is in registers: the next item's first P_bar V may overwrite it
       tc_fence_before();
       mbar_arrive(&o_free[t]);
-      if (row < p.N) {
+      if constexpr (L::kSepP) {
+        // each warp stages its 32 rows (128-byte swizzle) and lane 0 stores
+        // them with one TMA box; rows past N are clipped by the tensor map
+        uint8_t* stg = smem + L::kOOff + t * L::kTileBytes + (warp & 3) * 4096;
+        if (lane == 0) bulk_wait_read<0>();        // this warp's previous store has read the box
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+              make_uint4(ow[4 * c], ow[4 * c + 1], ow[4 * c + 2], ow[4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tm_o, stg, 0, w.q0_row + qt * 128 + (warp & 3) * 32, w.bh);
+          bulk_commit();
+        }
+      } else if (row < p.N) {
         uint4* dst = reinterpret_cast<uint4*>(static_cast<typename E::T*>(p.o) + (size_t(w.bh) * p.N + row) * D);
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(ow[4 * i], ow[4 * i + 1], ow[4 * i + 2], ow[4 * i + 3]);
+      }
+      if (row < p.N) {
         p.lse[size_t(w.bh) * p.N + row] = (ms + (raised ? p.delta_log2 : 0.f) + lg2(l)) * kLn2;
         if (kVariants && p.ties)
           p.ties[size_t(w.bh) * p.N + row] = cnt | (raised ? (1 << 29) : 0) | (ever_repeated ? (1 << 30) : 0);
@@ -650,6 +676,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       it_cnt += n_t;
     }
+    if (L::kSepP && lane == 0) bulk_wait<0>();     // every O store has landed
   }
 
   tc_fence_before();
