@@ -304,9 +304,10 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse,
   const size_t rows = size_t(BH) * N;
   const int BHkv = B * Hkv;
   constexpr CUtensorMapDataType dt = map_type<E>();
-  CUtensorMap mq, mk, mv, mdo, mdq;
+  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
   if (!make_map(&mq, q, BH, N, d, dt) || !make_map(&mk, k, BHkv, N, d, dt) || !make_map(&mv, v, BHkv, N, d, dt) ||
-      !make_map(&mdo, dout, BH, N, d, dt) || !make_map_dq(&mdq, workspace, BH, N, d))
+      !make_map(&mdo, dout, BH, N, d, dt) || !make_map_dq(&mdq, workspace, BH, N, d) ||
+      !make_map(&mdk, dk, BHkv, N, d, dt, 32) || !make_map(&mdv, dv, BHkv, N, d, dt, 32))
     return FA_ERR_DEVICE;
   BwdParams prm{};
   prm.lse = lse;
@@ -336,7 +337,7 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse,
   auto kern = (d == 64) ? (pairs ? fa_bwd_kernel<64, E, true> : fa_bwd_kernel<64, E, false>)
                         : (pairs ? fa_bwd_kernel<128, E, true> : fa_bwd_kernel<128, E, false>);
   const int smem = (d == 64) ? BwdLayout<64>::kAlloc : BwdLayout<128>::kAlloc;
-  const cudaError_t e = launch(kern, grid, dim3(BwdLayout<64>::kThreads), smem, s, mq, mk, mv, mdo, mdq, prm);
+  const cudaError_t e = launch(kern, grid, dim3(BwdLayout<64>::kThreads), smem, s, mq, mk, mv, mdo, mdq, mdk, mdv, prm);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 

@@ -221,6 +221,7 @@ struct BwdSteps {
 //               w%4) and queries 64*(w/4).. of each tile: P^T, dS^T
 //   warps 8-11  dQ drain (thread r owns query r; TMA reduce-add of 32 x 32
 //               FP32 boxes staged in shared memory) and the dK/dV epilogue
+//               (d = 64: through the same staging boxes and TMA stores)
 //   warp  12    producer: K, V per item; Q_i (TMA) plus LSE_i, D_i per step,
 //               up to kQStages steps ahead
 //   warp  14    producer: dO_i (TMA), independent of the Q ring
@@ -238,7 +239,8 @@ template <int D, typename E = ElemBF16, bool kPairs = false>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
+                  const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
   using L = BwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
@@ -714,29 +716,70 @@ __global__ void __launch_bounds__(512, 1)
       if (!ok) break;
       tc_fence_after();
       const int key = w.key0 + rr;
+      if constexpr (D == 64) {
+        // dV and dK through this warp's two staging boxes (32 rows each, the
+        // 128-byte swizzle) and one TMA store box each; rows past N are
+        // dropped by the tensor maps.  dV goes into the box the next dQ drain
+        // writes first, whose last reader is then the older of the two stores.
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t t_src = tmem + lane_base + (which ? L::kTmDK : L::kTmDV);
-        const float mul = which ? p.scale : 1.f;
-        uint32_t ov[D / 2];
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t t_src = tmem + lane_base + (which ? L::kTmDK : L::kTmDV);
+          const float mul = which ? p.scale : 1.f;
+          uint32_t r[2][32];
+          tmem_ld32(t_src, r[0]);
+          tmem_ld32(t_src + 32, r[1]);
+          tmem_ld_wait(r[0]);
+          tmem_ld_wait(r[1]);
+          if (which == 1) {
+            tc_fence_before();
+            mbar_arrive(dkv_free);                   // the next item may overwrite dK, dV
+          }
+          uint8_t* box = stage + ((box_seq + which) & 1) * L::kStageBox;
+          if (lane == 0) bulk_wait_read<1>();        // the group that last read this box is done reading
+          __syncwarp();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_src + c * 32, r);
-          tmem_ld_wait(r);
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            ov[c * 16 + i] = E::pack(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
+          for (int c = 0; c < 8; ++c) {
+            const int h = c >> 2, i0 = (c & 3) * 8;
+            uint4 v;
+            v.x = E::pack(__uint_as_float(r[h][i0 + 0]) * mul, __uint_as_float(r[h][i0 + 1]) * mul);
+            v.y = E::pack(__uint_as_float(r[h][i0 + 2]) * mul, __uint_as_float(r[h][i0 + 3]) * mul);
+            v.z = E::pack(__uint_as_float(r[h][i0 + 4]) * mul, __uint_as_float(r[h][i0 + 5]) * mul);
+            v.w = E::pack(__uint_as_float(r[h][i0 + 6]) * mul, __uint_as_float(r[h][i0 + 7]) * mul);
+            *reinterpret_cast<uint4*>(box + lane * 128 + ((c ^ (lane & 7)) << 4)) = v;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(which ? &tm_dk : &tm_dv, box, 0, w.key0 + wq * 32, w.bh);
+            bulk_commit();
+          }
         }
-        if (which == 1) {
-          tc_fence_before();
-          mbar_arrive(dkv_free);                     // the next item may overwrite dK, dV
-        }
-        if (key < p.N) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<typename E::T*>(which ? p.dk : p.dv) +
-                                                (size_t(w.bh) * p.N + key) * D);
-#pragma unroll
-          for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
+        box_seq += 2;
+      } else {
+  #pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t t_src = tmem + lane_base + (which ? L::kTmDK : L::kTmDV);
+          const float mul = which ? p.scale : 1.f;
+          uint32_t ov[D / 2];
+  #pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(t_src + c * 32, r);
+            tmem_ld_wait(r);
+  #pragma unroll
+            for (int i = 0; i < 16; ++i)
+              ov[c * 16 + i] = E::pack(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
+          }
+          if (which == 1) {
+            tc_fence_before();
+            mbar_arrive(dkv_free);                     // the next item may overwrite dK, dV
+          }
+          if (key < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<typename E::T*>(which ? p.dk : p.dv) +
+                                                  (size_t(w.bh) * p.N + key) * D);
+  #pragma unroll
+            for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
+          }
         }
       }
     }
