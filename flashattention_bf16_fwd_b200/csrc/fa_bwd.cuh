@@ -566,29 +566,42 @@ __global__ void __launch_bounds__(512, 1)
           tmem_ld_wait(r[0]);
           tmem_ld_wait(r[1]);
           const bool diag = p.causal && qt == w.kv_tile;
+          if (!__any_sync(0xffffffffu, !key_in || diag)) {   // no masked entry in this warp
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {               // 4 queries per shared-memory load of -LSE2
-            const float4 nl = *reinterpret_cast<const float4*>(nlse + 4 * j);
+            for (int j = 0; j < 16; ++j) {             // 4 queries per shared-memory load of -LSE2
+              const float4 nl = *reinterpret_cast<const float4*>(nlse + 4 * j);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int i = 2 * j + h;                 // pair of queries 2i, 2i+1 of this half
-              float x0, x1;
-              f2_unpack(f2_fma(f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
-                                       __uint_as_float(r[i >> 4][(2 * i + 1) & 31])),
-                               c2, h ? f2_pack(nl.z, nl.w) : f2_pack(nl.x, nl.y)),
-                        x0, x1);
-              pk[i] = E::pack(ex2(x0), ex2(x1));
+              for (int h = 0; h < 2; ++h) {
+                const int i = 2 * j + h;               // pair of queries 2i, 2i+1 of this half
+                float x0, x1;
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
+                                         __uint_as_float(r[i >> 4][(2 * i + 1) & 31])),
+                                 c2, h ? f2_pack(nl.z, nl.w) : f2_pack(nl.x, nl.y)),
+                          x0, x1);
+                pk[i] = E::pack(ex2(x0), ex2(x1));
+              }
             }
-          }
-          // masked keys (past N) and, on the diagonal tile, queries before the
-          // key: zero the packed halves (the warp takes this branch together)
-          if (__any_sync(0xffffffffu, !key_in || diag)) {
+          } else {
+            // masked keys (past N) and, on the diagonal tile, queries before
+            // the key: the exponent is set to -inf, so P = 0 (selected
+            // alongside the exponentials; a separate pass that cleared the
+            // packed halves afterwards cost ~1600 cycles per diagonal step)
+            const int lim = key_in ? (diag ? kr - 64 * half : 0) : 64;   // queries q < lim are masked
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int qg = 64 * half + 2 * i;        // query within the tile
-              const uint32_t lo = (!key_in || (diag && qg < kr)) ? 0u : 0x0000ffffu;
-              const uint32_t hi = (!key_in || (diag && qg + 1 < kr)) ? 0u : 0xffff0000u;
-              pk[i] &= lo | hi;
+            for (int j = 0; j < 16; ++j) {
+              const float4 nl = *reinterpret_cast<const float4*>(nlse + 4 * j);
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int i = 2 * j + h;
+                float x0, x1;
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(r[i >> 4][(2 * i) & 31]),
+                                         __uint_as_float(r[i >> 4][(2 * i + 1) & 31])),
+                                 c2, h ? f2_pack(nl.z, nl.w) : f2_pack(nl.x, nl.y)),
+                          x0, x1);
+                x0 = (2 * i < lim) ? -__int_as_float(0x7f800000) : x0;
+                x1 = (2 * i + 1 < lim) ? -__int_as_float(0x7f800000) : x1;
+                pk[i] = E::pack(ex2(x0), ex2(x1));
+              }
             }
           }
         }
