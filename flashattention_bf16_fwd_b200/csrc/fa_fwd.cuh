@@ -17,7 +17,8 @@
 //   warps 0-3  softmax warpgroup 0 (thread r owns row r: TMEM lane r)
 //   warps 4-7  softmax warpgroup 1
 //   warp  8    TMA producer: an item's Q tiles, then a ring of K/V stages
-//   warp  9    TMEM allocator + tcgen05.mma issuer (single thread); at d = 64
+//   warp  9    TMEM allocator + tcgen05.mma issuer (the whole warp runs the
+//              issuing loop, one elected lane executes each MMA); at d = 64
 //              it issues warpgroup 0's MMAs only
 //   warp 10    d = 64: tcgen05.mma issuer of warpgroup 1 (idle at d = 128)
 //   warp 11    idle (it completes the third warpgroup)
@@ -249,7 +250,14 @@ __global__ void __launch_bounds__(384, 1)
       // K/V stages are released once both issuers are done with them (their
       // empty barriers count two arrivals); a warpgroup whose tile of an item
       // is shorter goes on to the next item while the other finishes.
-      if (lane == 0) {
+      {
+        // The whole warp runs the loop (warp-uniform operands and waits); one
+        // elected lane executes each MMA.  From lane 0 alone, a tile's eight
+        // P_bar V MMAs took 600-1100 cycles to issue, which delayed the end
+        // of every item.
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+          return __all_sync(0xffffffffu, mbar_wait(bar, parity, wd));
+        };
         const int t = warp - 9;
         constexpr uint32_t kIdS = make_idesc(128, 128, 0, 0, E::kMmaFmt);
         constexpr uint32_t kIdPV = make_idesc(128, D, 0, 1, E::kMmaFmt);
@@ -263,17 +271,17 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t off = (k >> 2) * L::kSubBytes + (k & 3) * 32;
-            umma_ss(tmem + L::tm_s(t), sdesc_add(a, off), sdesc_add(b, off), kIdS, k > 0);
+            umma_ss_warp(tmem + L::tm_s(t), sdesc_add(a, off), sdesc_add(b, off), kIdS, k > 0);
           }
-          umma_commit(&s_full[t]);
+          umma_commit_warp(&s_full[t]);
         };
         auto issue_pv = [&](uint32_t st, int j) {
           const uint64_t b = sdesc_add(dv0, st * 2 * L::kTileBytes);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts(tmem + L::tm_o(t), tmem + L::tm_p(t) + k * 8, sdesc_add(b, k * 2048), kIdPV,
-                    (j > 0 || k > 0) ? 1u : 0u);
-          umma_commit(&o_done[t]);
+            umma_ts_warp(tmem + L::tm_o(t), tmem + L::tm_p(t) + k * 8, sdesc_add(b, k * 2048), kIdPV,
+                         (j > 0 || k > 0) ? 1u : 0u);
+          umma_commit_warp(&o_done[t]);
         };
         uint32_t kv_cnt = 0, it_cnt = 0, ep_cnt = 0, n_done = 0;
         bool ok = true;
@@ -281,28 +289,28 @@ __global__ void __launch_bounds__(384, 1)
           const FwdItem w = fwd_item(p, item);
           const int nt = fwd_tile_of<D>(t, rnd) ? w.n1 : w.n0;   // key tiles of this warpgroup's query tile
           qb = n_done % L::kQBufs;
-          if (!(ok = mbar_wait(&q_full[qb], (n_done / L::kQBufs) & 1, wd))) break;
+          if (!(ok = wait(&q_full[qb], (n_done / L::kQBufs) & 1))) break;
           if (nt > 0) {
-            if (!(ok = mbar_wait(&kv_full[kv_cnt % L::kStages], (kv_cnt / L::kStages) & 1, wd))) break;
-            if (it_cnt > 0 && !(ok = mbar_wait(&s_free[t], (it_cnt - 1) & 1, wd))) break;
+            if (!(ok = wait(&kv_full[kv_cnt % L::kStages], (kv_cnt / L::kStages) & 1))) break;
+            if (it_cnt > 0 && !(ok = wait(&s_free[t], (it_cnt - 1) & 1))) break;
             tc_fence_after();
             issue_s(kv_cnt % L::kStages);
           }
-          if (nt <= 1) umma_commit(&q_empty[qb]);   // this issuer's S MMAs of the item are issued
+          if (nt <= 1) umma_commit_warp(&q_empty[qb]);     // this issuer's S MMAs of the item are issued
           for (int j = 0; ok && j < w.nmax; ++j) {
             const uint32_t st = (kv_cnt + j) % L::kStages;
             if (j + 1 < nt) {
               const uint32_t nxt = kv_cnt + j + 1;
-              if (!(ok = mbar_wait(&kv_full[nxt % L::kStages], (nxt / L::kStages) & 1, wd) &&
-                         mbar_wait(&s_free[t], (it_cnt + j) & 1, wd)))
+              if (!(ok = wait(&kv_full[nxt % L::kStages], (nxt / L::kStages) & 1) &&
+                         wait(&s_free[t], (it_cnt + j) & 1)))
                 break;
               tc_fence_after();
               issue_s(nxt % L::kStages);
-              if (j + 2 == nt) umma_commit(&q_empty[qb]);
+              if (j + 2 == nt) umma_commit_warp(&q_empty[qb]);
             }
             if (j < nt) {
-              if (!(ok = mbar_wait(&p_full[t], (it_cnt + j) & 1, wd))) break;
-              if (j == 0 && !(ok = mbar_wait(&o_free[t], (ep_cnt & 1) ^ 1, wd))) break;
+              if (!(ok = wait(&p_full[t], (it_cnt + j) & 1))) break;
+              if (j == 0 && !(ok = wait(&o_free[t], (ep_cnt & 1) ^ 1))) break;
               tc_fence_after();
               issue_pv(st, j);
             }
@@ -310,23 +318,27 @@ __global__ void __launch_bounds__(384, 1)
             // fewer): wait until it is loaded before releasing its stage, so
             // that this issuer's arrival belongs to this use of the stage and
             // it never runs a use ahead of the other issuer
-            if (j >= nt && !(ok = mbar_wait(&kv_full[st], ((kv_cnt + j) / L::kStages) & 1, wd))) break;
-            umma_commit(&kv_empty[st]);          // this issuer is done with the stage
+            if (j >= nt && !(ok = wait(&kv_full[st], ((kv_cnt + j) / L::kStages) & 1))) break;
+            umma_commit_warp(&kv_empty[st]);     // this issuer is done with the stage
           }
           kv_cnt += w.nmax;
           it_cnt += nt;
           ep_cnt += (nt > 0) ? 1 : 0;
         }
-        umma_commit(&mma_done[t]);
-        mbar_wait(&mma_done[t], 0, wd);
+        umma_commit_warp(&mma_done[t]);
+        wait(&mma_done[t], 0);
       }
       __syncwarp();
-    } else if (warp == 9) {
-      // ---------------------------------------- d = 128: MMA issuer (one thread)
+    } else if (!L::kSepP && warp == 9) {
+      // ------------------------------------------------- d = 128: MMA issuer
       // Per key tile j: P_bar_0 V, S_0 of tile j+1 (it overwrites P_bar_0),
       // P_bar_1 V, S_1 of tile j+1; the two warpgroups alternate at the
       // tensor core.
-      if (lane == 0) {
+      {
+        // the whole warp runs the loop; one elected lane executes each MMA
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+          return __all_sync(0xffffffffu, mbar_wait(bar, parity, wd));
+        };
         constexpr uint32_t kIdS = make_idesc(128, 128, 0, 0, E::kMmaFmt);   // Q K^T: both K-major
         constexpr uint32_t kIdPV = make_idesc(128, D, 0, 1, E::kMmaFmt);    // P_bar V: V is MN-major
         // Descriptors are built once; each MMA only advances the start address.
@@ -339,17 +351,17 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t off = (k >> 2) * L::kSubBytes + (k & 3) * 32;
-            umma_ss(tmem + L::tm_s(t), sdesc_add(a, off), sdesc_add(b, off), kIdS, k > 0);
+            umma_ss_warp(tmem + L::tm_s(t), sdesc_add(a, off), sdesc_add(b, off), kIdS, k > 0);
           }
-          umma_commit(&s_full[t]);
+          umma_commit_warp(&s_full[t]);
         };
         auto issue_pv = [&](int t, uint32_t st, int j) {
           const uint64_t b = sdesc_add(dv0, st * 2 * L::kTileBytes);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts(tmem + L::tm_o(t), tmem + L::tm_p(t) + k * 8, sdesc_add(b, k * 2048), kIdPV,
-                    (j > 0 || k > 0) ? 1u : 0u);
-          umma_commit(&o_done[t]);
+            umma_ts_warp(tmem + L::tm_o(t), tmem + L::tm_p(t) + k * 8, sdesc_add(b, k * 2048), kIdPV,
+                         (j > 0 || k > 0) ? 1u : 0u);
+          umma_commit_warp(&o_done[t]);
         };
         uint32_t kv_cnt = 0;           // K/V tiles consumed
         uint32_t it_cnt[2] = {0, 0};   // softmax iterations per query tile
@@ -359,35 +371,35 @@ __global__ void __launch_bounds__(384, 1)
         for (int rnd = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++rnd), ++n_done) {
           const FwdItem w = fwd_item(p, item);
           const int nt[2] = {w.n0, w.n1};
-          if (!(ok = mbar_wait(q_full, n_done & 1, wd) &&
-                     mbar_wait(&kv_full[kv_cnt % L::kStages], (kv_cnt / L::kStages) & 1, wd)))
+          if (!(ok = wait(q_full, n_done & 1) &&
+                     wait(&kv_full[kv_cnt % L::kStages], (kv_cnt / L::kStages) & 1)))
             break;
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
             if (nt[t] > 0) issue_s(t, kv_cnt % L::kStages);
-          if (w.nmax == 1) umma_commit(q_empty);
+          if (w.nmax == 1) umma_commit_warp(q_empty);
           for (int j = 0; ok && j < w.nmax; ++j) {
             const uint32_t st = (kv_cnt + j) % L::kStages;
             const uint32_t stn = (kv_cnt + j + 1) % L::kStages;
             for (int t = 0; t < 2; ++t) {
               if (j < nt[t]) {
-                if (!(ok = mbar_wait(&p_full[t], (it_cnt[t] + j) & 1, wd))) break;
+                if (!(ok = wait(&p_full[t], (it_cnt[t] + j) & 1))) break;
                 // the first P_bar V of an item overwrites O_t: the previous
                 // item's epilogue must have read it
-                if (j == 0 && !(ok = mbar_wait(&o_free[t], (ep_cnt[t] & 1) ^ 1, wd))) break;
+                if (j == 0 && !(ok = wait(&o_free[t], (ep_cnt[t] & 1) ^ 1))) break;
                 tc_fence_after();
                 issue_pv(t, st, j);
               }
               if (t == 0 && j + 1 < w.nmax) {
                 const uint32_t nxt = kv_cnt + j + 1;
-                if (!(ok = mbar_wait(&kv_full[stn], (nxt / L::kStages) & 1, wd))) break;
+                if (!(ok = wait(&kv_full[stn], (nxt / L::kStages) & 1))) break;
                 tc_fence_after();
                 if (j + 1 < nt[0]) issue_s(0, stn);   // S_0 of tile j+1 overwrites P_bar_0 after P_bar V
               }
               if (t == 1) {
-                umma_commit(&kv_empty[st]);
+                umma_commit_warp(&kv_empty[st]);
                 if (j + 1 < nt[1]) issue_s(1, stn);
-                if (j + 2 == w.nmax) umma_commit(q_empty);   // the item's last S MMAs are issued
+                if (j + 2 == w.nmax) umma_commit_warp(q_empty);   // the item's last S MMAs are issued
               }
             }
           }
@@ -398,8 +410,8 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         // Every MMA must be finished before TMEM is released.
-        umma_commit(&mma_done[0]);
-        mbar_wait(&mma_done[0], 0, wd);
+        umma_commit_warp(&mma_done[0]);
+        wait(&mma_done[0], 0);
       }
       __syncwarp();
     }

@@ -318,6 +318,28 @@ __device__ __forceinline__ void umma_ts_lh_warp(uint32_t d_tmem, uint32_t a_tmem
       : "memory");
 }
 
+__device__ __forceinline__ void umma_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred P, E;\n\t"
+      "elect.sync _|E, 0xffffffff;\n\t"
+      "setp.ne.b32 P, %4, 0;\n\t"
+      "@E tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, P;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred P, E;\n\t"
+      "elect.sync _|E, 0xffffffff;\n\t"
+      "setp.ne.b32 P, %4, 0;\n\t"
+      "@E tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, P;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred E;\n\t"
