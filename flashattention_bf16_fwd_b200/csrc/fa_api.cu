@@ -290,7 +290,7 @@ int pre_impl(const void* o, const void* dout, void* workspace, size_t workspace_
 template <typename E>
 int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse, const void* dout, void* dk, void* dv,
                   void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N, int d, int causal,
-                  float scale, void* stream) {
+                  float scale, void* stream, bool after_pre = false) {
   if (!q || !k || !v || !lse || !dout || !dk || !dv) return FA_ERR_NULL;
   int rc = check_common(B, H, N, d, causal, scale);
   if (rc != FA_OK) return rc;
@@ -331,6 +331,7 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse,
   prm.causal = causal;
   prm.scale = scale;
   prm.scale_log2 = float(double(scale) * 1.4426950408889634);
+  prm.after_pre = after_pre ? 1 : 0;
   const int n_items = prm.n_kv * BHkv;
   const dim3 grid(unsigned(n_items < st->num_sms ? n_items : st->num_sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -378,8 +379,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   (void)st;
   rc = pre_impl<E>(o, dout, workspace, workspace_bytes, B, H, N, d, stream);
   if (rc != FA_OK) return rc;
+  // launched right after the preprocess: it may start its input loads early
   rc = bwd_main_impl<E>(q, k, v, lse, dout, dk, dv, workspace, workspace_bytes, B, H, Hkv, N, d, causal, scale,
-                        stream);
+                        stream, true);
   if (rc != FA_OK) return rc;
   return finish_impl<E>(dq, workspace, workspace_bytes, B, H, N, d, scale, stream);
 }

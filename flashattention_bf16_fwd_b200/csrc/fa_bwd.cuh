@@ -88,6 +88,7 @@ struct BwdParams {
   int BH, N, n_kv, causal;   // BH = batch * K/V heads
   int H, group;         // query heads per batch entry; query heads per K/V head (1 = no sharing)
   float scale, scale_log2;
+  int after_pre;        // 1: launched right after fa_bwd_pre_kernel on the same stream
 };
 
 template <int D>
@@ -310,9 +311,14 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // set-up above touched no global memory; from here on the previous
-  // kernel's writes are needed
-  grid_dep_wait();
+  // Set-up above touched no global memory.  Launched right after the
+  // preprocess kernel (after_pre), which let this kernel start only once every
+  // kernel before it had finished, Q, K, V, dO and LSE are complete here and
+  // only D and the zeroed dQ accumulator are not: then only the threads that
+  // read D (the Q producer) or write global memory (the dQ drain and the
+  // dK/dV epilogue) wait for the preprocess, and the K, V, Q and dO loads and
+  // the first S and dP MMAs overlap its end.  Otherwise every thread waits.
+  if (!p.after_pre) grid_dep_wait();
   grid_dep_launch();
   const Watchdog wd{abort_flag, p.dev_error};
 
@@ -327,6 +333,7 @@ __global__ void __launch_bounds__(512, 1)
       uint32_t g = 0;        // query-tile steps loaded
       uint32_t n_done = 0;   // items started
       bool ok = true;
+      bool dep_done = false;
       for (BwdSched<kPairs> sc(p); ok && sc.valid(); sc.next(p), ++n_done) {
         const BwdItem w = sc.get(p);
         const uint32_t ks = n_done % L::kKVStages;
@@ -352,6 +359,10 @@ __global__ void __launch_bounds__(512, 1)
             for (int s = 0; s < L::kSub; ++s)
               tma_load_3d(smem + L::kQOff + st * L::kTileBytes + s * L::kSubBytes, &tm_q, &q_full[st], s * 64, q0,
                           sp.bh_q, pol_q);
+          }
+          if (!dep_done) {                     // D comes from the preprocess kernel
+            grid_dep_wait();
+            dep_done = true;
           }
           float* nlse = stats + st * 256;
           float* dd = nlse + 128;
@@ -672,6 +683,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else {
     regs_set<L::kDrainRegs, L::kLaunchRegs>();
+    grid_dep_wait();                                   // the preprocess zeroes the dQ accumulator
     // ------------------------------------------- dQ drain and dK/dV epilogue
     const int wq = warp & 3;
     const int rr = wq * 32 + lane;                   // query row (dQ) / key row (dK, dV)
