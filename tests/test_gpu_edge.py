@@ -153,3 +153,41 @@ def test_forward_repeats_bit_for_bit(fa, B, H, N, d, causal):
     torch.cuda.synchronize()
     assert fa.fa_check_device_error() == 0
     assert torch.equal(p0[0], o0) and torch.equal(p0[1], l0)
+
+
+SPLIT_CASES = [(2, 3, 777, 64, True), (1, 4, 1000, 64, True), (2, 2, 700, 128, True), (1, 3, 333, 64, False)]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", SPLIT_CASES,
+                         ids=[f"B{b}H{h}N{n}d{d}{'c' if c else 'f'}" for b, h, n, d, c in SPLIT_CASES])
+def test_backward_one_call_matches_three_calls(fa, B, H, N, d, causal):
+    """fa_bwd launches the main kernel right after the preprocess and lets it
+    load Q, K, V, dO and LSE and start its first MMAs before the preprocess
+    has finished (only D and the zeroed dQ accumulator come from it); the
+    three calls one by one make every thread of the main kernel wait.  Both
+    give the same dK and dV bit for bit (each is summed in one CTA in a fixed
+    order) and the same dQ up to the order of the FP32 reduce-adds, repeated
+    20 times so that a read of D or of the accumulator ahead of the
+    preprocess would show (the workspace holds NaN before each call)."""
+    x = make_inputs(Workload("split", B, H, N, d, causal=causal), seed=N + d + 7 * B)
+    dev = torch.device("cuda")
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, lse = fa.attention_fwd(q, k, v, causal=causal, scale=x["scale"], fix_mode=1)
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    dq3, dk3, dv3 = (torch.empty_like(q) for _ in range(3))
+    for call, rc in (("pre", fa.fa_bwd_preprocess(o, do, ws)),
+                     ("main", fa.fa_bwd_main(q, k, v, lse, do, dk3, dv3, ws, causal, x["scale"])),
+                     ("finish", fa.fa_bwd_finish(dq3, ws, x["scale"]))):
+        assert rc == 0, call
+    torch.cuda.synchronize()
+    assert fa.fa_check_device_error() == 0
+    for _ in range(20):
+        dq1, dk1, dv1 = (torch.empty_like(q) for _ in range(3))
+        ws.fill_(0xFF)                                 # NaN in D and in the accumulator until the preprocess runs
+        assert fa.fa_bwd(q, k, v, o, lse, do, dq1, dk1, dv1, ws, causal, x["scale"]) == 0
+        torch.cuda.synchronize()
+        assert fa.fa_check_device_error() == 0
+        assert torch.equal(dk1, dk3) and torch.equal(dv1, dv3)
+        # dQ: FP32 sums in a varying order, then one rounding to bf16
+        diff = (dq1.float() - dq3.float()).abs()
+        assert float(diff.max()) <= 2 ** -7 * float(dq3.float().abs().max()) + 1e-6
