@@ -318,6 +318,7 @@ __device__ __forceinline__ void umma_ts_lh_warp(uint32_t d_tmem, uint32_t a_tmem
       : "memory");
 }
 
+// Whole-warp issue with full 64-bit descriptors (the forward's issuers).
 __device__ __forceinline__ void umma_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                              uint32_t accumulate) {
   asm volatile(
