@@ -506,7 +506,7 @@ def measure_config(fa, w, args, rank, dev, stream, flush):
 
 
 def measured_traffic(kernel, w):
-    """DRAM bytes per launch from the committed ncu capture, if it matches this kernel build."""
+    """DRAM bytes per launch from the committed ncu capture of this workload, if it matches this kernel build."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -525,9 +525,8 @@ def measured_traffic(kernel, w):
             h.update(f.read())
     if rec.get("csrc_sha256") != h.hexdigest():
         return None
-    if rec.get("workload") != w.name:
-        return None
-    return rec.get("dram_bytes_per_launch")
+    per = rec.get("per_workload", {}).get(w.name)
+    return per.get("dram_bytes_per_launch") if per else None
 
 
 def run_e2e(fa, x, w, args, dev, stream, flops_total, world):

@@ -83,3 +83,26 @@ def test_max_over_ranks_gloo():
         t_max, value = res[rank]
         assert t_max == 1500.0                   # every rank sees the slowest rank's time
         assert value == pytest.approx(world * 10 * 1e12 / 1.5 / 1e12)
+
+
+def test_measured_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
+    """The roofline's DRAM traffic comes from the committed ncu record only
+    while the kernel's sources hash to the value stored with it, and only for
+    the workload it was captured on."""
+    import hashlib
+    from flashattention_bf16_fwd_b200.workloads import WORKLOADS
+    src = tmp_path / "flashattention_bf16_fwd_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "a.cuh").write_text("kernel A\n")
+    (src / "b.cuh").write_text("helpers\n")
+    digest = hashlib.sha256(b"kernel A\nhelpers\n").hexdigest()
+    (tmp_path / "profiles").mkdir()
+    rec = {"fa_bwd_kernel": {"sources": ["a.cuh", "b.cuh"], "csrc_sha256": digest,
+                             "per_workload": {"gpt2s": {"dram_bytes_per_launch": 1234}}}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("fa_bwd_kernel", WORKLOADS["gpt2s"]) == 1234
+    assert bench.measured_traffic("fa_bwd_kernel", WORKLOADS["gpt2m"]) is None
+    assert bench.measured_traffic("fa_fwd_kernel", WORKLOADS["gpt2s"]) is None
+    (src / "b.cuh").write_text("helpers, changed\n")
+    assert bench.measured_traffic("fa_bwd_kernel", WORKLOADS["gpt2s"]) is None
